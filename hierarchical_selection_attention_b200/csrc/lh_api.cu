@@ -1,0 +1,407 @@
+// C ABI of the Lighthouse Attention hot path (declared in lighthouse.h):
+// argument checking, buffer layouts and the order of the launches.  No
+// arithmetic of the method lives here.
+#include <math.h>
+#include <string.h>
+
+#include "lh_common.cuh"
+
+namespace {
+
+__device__ int g_status_word[2];  // [code, detail], see lh_get_device_status
+
+constexpr size_t kAlign = 256;
+inline size_t up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+
+int* status_ptr() {
+  static int* ptrs[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int*>(p);
+  }
+  return ptrs[dev];
+}
+
+lh_status check(const lh_config* c) {
+  if (!c) return LH_ERR_INVALID_ARGUMENT;
+  if (c->B < 1 || c->N < 1 || c->H < 1 || c->p < 2 || c->L < 1 || c->k < 0)
+    return LH_ERR_INVALID_ARGUMENT;
+  if (c->L > 6) return LH_ERR_UNSUPPORTED;
+  if (c->N >= (1LL << 31) || c->H >= (1 << 16) || c->B >= (1 << 16)) return LH_ERR_UNSUPPORTED;
+  int64_t w = 1;
+  for (int l = 1; l < c->L; ++l) {
+    if (w > c->N / c->p) return LH_ERR_INVALID_ARGUMENT;  // p^(L-1) > N
+    w *= c->p;
+  }
+  if (c->N % w) return LH_ERR_INVALID_ARGUMENT;  // Sec. 3.3: p^(L-1) | N
+  int64_t cand = 0, P = 0, span = 1;
+  for (int l = 0; l < c->L; ++l) {
+    P += c->N / span;
+    if (l < c->L - 1) cand += c->N / span;
+    span *= (l < c->L - 1) ? c->p : 1;
+  }
+  if (c->k > (1LL << 31)) return LH_ERR_INVALID_ARGUMENT;
+  const int64_t n_sel = (c->L - 1) * c->p * c->k;
+  if (n_sel > cand) return LH_ERR_INVALID_ARGUMENT;
+  if (P >= (1LL << 31)) return LH_ERR_UNSUPPORTED;
+  if (c->d != 64 && c->d != 128) return LH_ERR_UNSUPPORTED;
+  if (c->scatter_mode != 0 && c->scatter_mode != 1) return LH_ERR_INVALID_ARGUMENT;
+  if (c->select_mode != 0) return LH_ERR_UNSUPPORTED;
+  if (!(c->scale == c->scale)) return LH_ERR_INVALID_ARGUMENT;
+  const int64_t S = c->N / w + n_sel;
+  if (S >= (1LL << 31) || (int64_t)c->B * c->H * ((S + 127) / 128) >= (1LL << 31))
+    return LH_ERR_UNSUPPORTED;
+  return LH_OK;
+}
+
+LhDims dims(const lh_config* c) {
+  LhDims D;
+  memset(&D, 0, sizeof(D));
+  D.B = (int)c->B; D.H = (int)c->H; D.d = (int)c->d; D.L = (int)c->L; D.p = (int)c->p;
+  D.N = c->N;
+  int64_t span = 1, off = 0, prow = 0;
+  for (int l = 0; l < D.L; ++l) {
+    D.lvl_span[l] = span;
+    D.lvl_size[l] = c->N / span;
+    D.lvl_off[l] = off;
+    D.pool_row[l] = l == 0 ? 0 : prow;
+    if (l >= 1) prow += D.lvl_size[l];
+    off += D.lvl_size[l];
+    span *= c->p;
+  }
+  D.P = off;
+  D.pooled_rows = prow;
+  D.n_cand = D.L > 1 ? D.lvl_off[D.L - 1] : 0;
+  D.n_sel = (int64_t)(D.L - 1) * c->p * c->k;
+  D.S = D.lvl_size[D.L - 1] + D.n_sel;
+  D.scale = c->scale > 0.f ? c->scale : (float)(1.0 / sqrt((double)c->d));
+  D.status = nullptr;
+  return D;
+}
+
+// Dims for a call that launches kernels: adds the device status word.
+LhDims launch_dims(const lh_config* c) {
+  LhDims D = dims(c);
+  D.status = status_ptr();
+  return D;
+}
+
+struct FwdWs {
+  size_t select, q_lv, k_lv, v_lv, qk, kq, atomic, total;
+};
+
+FwdWs fwd_layout(const LhDims& D, int scatter_mode) {
+  FwdWs w;
+  const size_t pooled = (size_t)D.B * D.pooled_rows * D.H * D.d * 2;
+  const size_t sc = (size_t)D.B * D.H * D.P * 4;
+  size_t o = 0;
+  w.select = o; o += up(lh_select_ws_bytes(D));
+  w.q_lv = o; o += up(pooled);
+  w.k_lv = o; o += up(pooled);
+  w.v_lv = o; o += up(pooled);
+  w.qk = o; o += up(sc);
+  w.kq = o; o += up(sc);
+  w.atomic = o; o += scatter_mode == 1 ? up(lh_scatter_atomic_ws_bytes(D)) : 0;
+  w.total = o;
+  return w;
+}
+
+struct Saved {
+  size_t off[7];
+  size_t total;
+};
+
+Saved saved_layout(const LhDims& D) {
+  Saved s;
+  const size_t rows = (size_t)D.B * D.H * D.S;
+  const size_t sizes[7] = {rows * 4, (size_t)D.B * D.H * D.P * 4, rows * D.d * 2, rows * D.d * 2,
+                           rows * D.d * 2, rows * D.d * 2, rows * 4};
+  size_t o = 0;
+  for (int i = 0; i < 7; ++i) {
+    s.off[i] = o;
+    o += up(sizes[i]);
+  }
+  s.total = o;
+  return s;
+}
+
+struct BwdWs {
+  size_t dog, delta, dqg, dkg, dvg, total;
+};
+
+BwdWs bwd_layout(const LhDims& D) {
+  BwdWs b;
+  const size_t rows = (size_t)D.B * D.H * D.S;
+  size_t o = 0;
+  b.delta = o; o += up(rows * 4);
+  b.dog = o; o += up(rows * D.d * 2);
+  b.dqg = o; o += up(rows * D.d * 2);
+  b.dkg = o; o += up(rows * D.d * 2);
+  b.dvg = o; o += up(rows * D.d * 2);
+  b.total = o;
+  return b;
+}
+
+inline bool aligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+template <typename... Ts>
+inline bool all_aligned(Ts... ps) {
+  bool ok = true;
+  ((ok = ok && ps != nullptr && aligned(ps)), ...);
+  return ok;
+}
+
+inline lh_status cu(cudaError_t e) { return e == cudaSuccess ? LH_OK : LH_ERR_CUDA; }
+
+template <typename T>
+inline T* at(void* base, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(base) + off);
+}
+template <typename T>
+inline const T* at(const void* base, size_t off) {
+  return reinterpret_cast<const T*>(static_cast<const char*>(base) + off);
+}
+
+#define LH_TRY(expr)                   \
+  do {                                 \
+    lh_status _s = (expr);             \
+    if (_s != LH_OK) return _s;        \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+lh_status lh_config_check(const lh_config* cfg) { return check(cfg); }
+
+int64_t lh_subseq_len(const lh_config* cfg) {
+  if (check(cfg) != LH_OK) return -1;
+  return dims(cfg).S;
+}
+
+int64_t lh_total_entries(const lh_config* cfg) {
+  if (check(cfg) != LH_OK) return -1;
+  return dims(cfg).P;
+}
+
+int64_t lh_pooled_rows(const lh_config* cfg) {
+  if (check(cfg) != LH_OK) return -1;
+  return dims(cfg).pooled_rows;
+}
+
+lh_status lh_workspace_bytes(const lh_config* cfg, size_t* fwd_ws, size_t* bwd_ws,
+                             size_t* saved) {
+  LH_TRY(check(cfg));
+  const LhDims D = dims(cfg);
+  if (fwd_ws) *fwd_ws = fwd_layout(D, cfg->scatter_mode).total;
+  if (bwd_ws) *bwd_ws = bwd_layout(D).total;
+  if (saved) *saved = saved_layout(D).total;
+  return LH_OK;
+}
+
+lh_status lh_saved_offsets(const lh_config* cfg, size_t* offsets) {
+  LH_TRY(check(cfg));
+  if (!offsets) return LH_ERR_INVALID_ARGUMENT;
+  const Saved s = saved_layout(dims(cfg));
+  for (int i = 0; i < 7; ++i) offsets[i] = s.off[i];
+  return LH_OK;
+}
+
+lh_status lh_pyramid(const lh_config* cfg, const lh_bf16* q, const lh_bf16* k,
+                     const lh_bf16* v, lh_bf16* q_lv, lh_bf16* k_lv, lh_bf16* v_lv,
+                     float* qk, float* kq, void* stream) {
+  LH_TRY(check(cfg));
+  if (!all_aligned(q, k, v, qk, kq)) return LH_ERR_INVALID_ARGUMENT;
+  if (cfg->L > 1 && !all_aligned(q_lv, k_lv, v_lv)) return LH_ERR_INVALID_ARGUMENT;
+  const LhDims D = launch_dims(cfg);
+  if (!D.status) return LH_ERR_CUDA;
+  return cu(lh_launch_pyramid(D, q, k, v, q_lv, k_lv, v_lv, qk, kq, (cudaStream_t)stream));
+}
+
+lh_status lh_score_topk(const lh_config* cfg, const float* qk, const float* kq,
+                        int32_t* sel_idx, int32_t* slot_map, void* ws, size_t ws_bytes,
+                        void* stream) {
+  LH_TRY(check(cfg));
+  if (!all_aligned(qk, kq, sel_idx, slot_map, ws)) return LH_ERR_INVALID_ARGUMENT;
+  const LhDims D = launch_dims(cfg);
+  if (!D.status) return LH_ERR_CUDA;
+  if (ws_bytes < lh_select_ws_bytes(D)) return LH_ERR_WORKSPACE;
+  return cu(lh_launch_select(D, qk, kq, sel_idx, slot_map, ws, (cudaStream_t)stream, nullptr));
+}
+
+lh_status lh_gather(const lh_config* cfg, const lh_bf16* q, const lh_bf16* k,
+                    const lh_bf16* v, const lh_bf16* q_lv, const lh_bf16* k_lv,
+                    const lh_bf16* v_lv, const int32_t* sel_idx, lh_bf16* qg, lh_bf16* kg,
+                    lh_bf16* vg, void* stream) {
+  LH_TRY(check(cfg));
+  if (!all_aligned(q, k, v, sel_idx, qg, kg, vg)) return LH_ERR_INVALID_ARGUMENT;
+  if (cfg->L > 1 && !all_aligned(q_lv, k_lv, v_lv)) return LH_ERR_INVALID_ARGUMENT;
+  const LhDims D = launch_dims(cfg);
+  if (!D.status) return LH_ERR_CUDA;
+  return cu(lh_launch_gather(D, q, k, v, q_lv, k_lv, v_lv, sel_idx, qg, kg, vg,
+                             (cudaStream_t)stream));
+}
+
+lh_status lh_attn_fwd(const lh_config* cfg, const lh_bf16* qg, const lh_bf16* kg,
+                      const lh_bf16* vg, lh_bf16* og, float* lse, void* stream) {
+  LH_TRY(check(cfg));
+  if (!all_aligned(qg, kg, vg, og, lse)) return LH_ERR_INVALID_ARGUMENT;
+  const LhDims D = launch_dims(cfg);
+  if (!D.status) return LH_ERR_CUDA;
+  return cu(lh_launch_attn_fwd(D.B * D.H, D.S, D.d, D.scale, qg, kg, vg, og, lse, D.status,
+                               (cudaStream_t)stream));
+}
+
+lh_status lh_attn_bwd(const lh_config* cfg, const lh_bf16* qg, const lh_bf16* kg,
+                      const lh_bf16* vg, const lh_bf16* og, const float* lse,
+                      const lh_bf16* dog, lh_bf16* dqg, lh_bf16* dkg, lh_bf16* dvg, void* ws,
+                      size_t ws_bytes, void* stream) {
+  LH_TRY(check(cfg));
+  if (!all_aligned(qg, kg, vg, og, lse, dog, dqg, dkg, dvg, ws)) return LH_ERR_INVALID_ARGUMENT;
+  const LhDims D = launch_dims(cfg);
+  if (!D.status) return LH_ERR_CUDA;
+  const BwdWs b = bwd_layout(D);
+  if (ws_bytes < b.total) return LH_ERR_WORKSPACE;
+  const cudaStream_t st = (cudaStream_t)stream;
+  float* delta = at<float>(ws, b.delta);
+  LH_TRY(cu(lh_launch_attn_delta(D.B * D.H, D.S, D.d, og, dog, delta, st)));
+  return cu(lh_launch_attn_bwd(D.B * D.H, D.S, D.d, D.scale, qg, kg, vg, dog, lse, delta, dqg,
+                               dkg, dvg, D.status, st, nullptr));
+}
+
+lh_status lh_scatter(const lh_config* cfg, const lh_bf16* og, const int32_t* slot_map,
+                     lh_bf16* o, void* ws, size_t ws_bytes, void* stream) {
+  LH_TRY(check(cfg));
+  if (!all_aligned(og, slot_map, o)) return LH_ERR_INVALID_ARGUMENT;
+  const LhDims D = launch_dims(cfg);
+  if (!D.status) return LH_ERR_CUDA;
+  if (cfg->scatter_mode == 1) {
+    if (!all_aligned(ws)) return LH_ERR_INVALID_ARGUMENT;
+    if (ws_bytes < lh_scatter_atomic_ws_bytes(D)) return LH_ERR_WORKSPACE;
+    return cu(lh_launch_scatter_atomic(D, og, slot_map, o, ws, (cudaStream_t)stream, nullptr));
+  }
+  return cu(lh_launch_scatter(D, og, slot_map, o, (cudaStream_t)stream));
+}
+
+lh_status lh_scatter_bwd(const lh_config* cfg, const lh_bf16* dout, const lh_bf16* og,
+                         const int32_t* sel_idx, lh_bf16* dog, float* delta, void* stream) {
+  LH_TRY(check(cfg));
+  if (!all_aligned(dout, og, sel_idx, dog, delta)) return LH_ERR_INVALID_ARGUMENT;
+  const LhDims D = launch_dims(cfg);
+  if (!D.status) return LH_ERR_CUDA;
+  return cu(lh_launch_scatter_bwd(D, dout, og, sel_idx, dog, delta, (cudaStream_t)stream));
+}
+
+lh_status lh_gather_bwd(const lh_config* cfg, const lh_bf16* dqg, const lh_bf16* dkg,
+                        const lh_bf16* dvg, const int32_t* slot_map, lh_bf16* dq, lh_bf16* dk,
+                        lh_bf16* dv, void* stream) {
+  LH_TRY(check(cfg));
+  if (!all_aligned(dqg, dkg, dvg, slot_map, dq, dk, dv)) return LH_ERR_INVALID_ARGUMENT;
+  const LhDims D = launch_dims(cfg);
+  if (!D.status) return LH_ERR_CUDA;
+  return cu(lh_launch_gather_bwd(D, dqg, dkg, dvg, slot_map, dq, dk, dv, (cudaStream_t)stream));
+}
+
+lh_status lh_forward(const lh_config* cfg, const lh_bf16* q, const lh_bf16* k,
+                     const lh_bf16* v, lh_bf16* o, void* saved, size_t saved_bytes, void* ws,
+                     size_t ws_bytes, void* stream) {
+  LH_TRY(check(cfg));
+  if (!all_aligned(q, k, v, o, saved, ws)) return LH_ERR_INVALID_ARGUMENT;
+  const LhDims D = launch_dims(cfg);
+  if (!D.status) return LH_ERR_CUDA;
+  const FwdWs w = fwd_layout(D, cfg->scatter_mode);
+  const Saved s = saved_layout(D);
+  if (ws_bytes < w.total || saved_bytes < s.total) return LH_ERR_WORKSPACE;
+  const cudaStream_t st = (cudaStream_t)stream;
+  int32_t* sel_idx = at<int32_t>(saved, s.off[0]);
+  int32_t* slot_map = at<int32_t>(saved, s.off[1]);
+  lh_bf16* qg = at<lh_bf16>(saved, s.off[2]);
+  lh_bf16* kg = at<lh_bf16>(saved, s.off[3]);
+  lh_bf16* vg = at<lh_bf16>(saved, s.off[4]);
+  lh_bf16* og = at<lh_bf16>(saved, s.off[5]);
+  float* lse = at<float>(saved, s.off[6]);
+  lh_bf16* q_lv = at<lh_bf16>(ws, w.q_lv);
+  lh_bf16* k_lv = at<lh_bf16>(ws, w.k_lv);
+  lh_bf16* v_lv = at<lh_bf16>(ws, w.v_lv);
+  float* qk = at<float>(ws, w.qk);
+  float* kq = at<float>(ws, w.kq);
+  LH_TRY(cu(lh_launch_pyramid(D, q, k, v, q_lv, k_lv, v_lv, qk, kq, st)));
+  LH_TRY(cu(lh_launch_select(D, qk, kq, sel_idx, slot_map, at<void>(ws, w.select), st, nullptr)));
+  LH_TRY(cu(lh_launch_gather(D, q, k, v, q_lv, k_lv, v_lv, sel_idx, qg, kg, vg, st)));
+  LH_TRY(cu(lh_launch_attn_fwd(D.B * D.H, D.S, D.d, D.scale, qg, kg, vg, og, lse, D.status, st)));
+  if (cfg->scatter_mode == 1)
+    return cu(lh_launch_scatter_atomic(D, og, slot_map, o, at<void>(ws, w.atomic), st, nullptr));
+  return cu(lh_launch_scatter(D, og, slot_map, o, st));
+}
+
+lh_status lh_backward(const lh_config* cfg, const void* saved, size_t saved_bytes,
+                      const lh_bf16* dout, lh_bf16* dq, lh_bf16* dk, lh_bf16* dv, void* ws,
+                      size_t ws_bytes, void* stream) {
+  LH_TRY(check(cfg));
+  if (!all_aligned(saved, dout, dq, dk, dv, ws)) return LH_ERR_INVALID_ARGUMENT;
+  const LhDims D = launch_dims(cfg);
+  if (!D.status) return LH_ERR_CUDA;
+  const Saved s = saved_layout(D);
+  const BwdWs b = bwd_layout(D);
+  if (saved_bytes < s.total || ws_bytes < b.total) return LH_ERR_WORKSPACE;
+  const cudaStream_t st = (cudaStream_t)stream;
+  const int32_t* sel_idx = at<int32_t>(saved, s.off[0]);
+  const int32_t* slot_map = at<int32_t>(saved, s.off[1]);
+  const lh_bf16* qg = at<lh_bf16>(saved, s.off[2]);
+  const lh_bf16* kg = at<lh_bf16>(saved, s.off[3]);
+  const lh_bf16* vg = at<lh_bf16>(saved, s.off[4]);
+  const lh_bf16* og = at<lh_bf16>(saved, s.off[5]);
+  const float* lse = at<float>(saved, s.off[6]);
+  lh_bf16* dog = at<lh_bf16>(ws, b.dog);
+  float* delta = at<float>(ws, b.delta);
+  lh_bf16* dqg = at<lh_bf16>(ws, b.dqg);
+  lh_bf16* dkg = at<lh_bf16>(ws, b.dkg);
+  lh_bf16* dvg = at<lh_bf16>(ws, b.dvg);
+  LH_TRY(cu(lh_launch_scatter_bwd(D, dout, og, sel_idx, dog, delta, st)));
+  LH_TRY(cu(lh_launch_attn_bwd(D.B * D.H, D.S, D.d, D.scale, qg, kg, vg, dog, lse, delta, dqg,
+                               dkg, dvg, D.status, st, nullptr)));
+  return cu(lh_launch_gather_bwd(D, dqg, dkg, dvg, slot_map, dq, dk, dv, st));
+}
+
+lh_status lh_get_device_status(void* stream, int32_t* detail) {
+  int* p = status_ptr();
+  if (!p) return LH_ERR_CUDA;
+  int h[2] = {0, 0};
+  const cudaStream_t st = (cudaStream_t)stream;
+  if (cudaMemcpyAsync(h, p, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess) return LH_ERR_CUDA;
+  if (cudaMemsetAsync(p, 0, sizeof(h), st) != cudaSuccess) return LH_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return LH_ERR_CUDA;
+  if (detail) *detail = h[1];
+  return (lh_status)h[0];
+}
+
+const char* lh_status_string(lh_status s) {
+  switch (s) {
+    case LH_OK: return "ok";
+    case LH_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case LH_ERR_UNSUPPORTED: return "unsupported configuration";
+    case LH_ERR_WORKSPACE: return "workspace or saved buffer too small";
+    case LH_ERR_CUDA: return "CUDA launch or driver error";
+    case LH_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case LH_ERR_DEVICE_BOUNDS: return "device-side index check failed";
+  }
+  return "unknown status";
+}
+
+int32_t lh_forward_launches(const lh_config* cfg) {
+  if (check(cfg) != LH_OK) return -1;
+  const LhDims D = dims(cfg);
+  const int select = D.n_cand > 0 ? 12 + 1 + 3 : 1 + 1 + 3;  // memset + hist/find pairs + order
+  const int scatter = cfg->scatter_mode == 1 ? 3 : 1;
+  return 1 + select + 1 + 1 + scatter;
+}
+
+int32_t lh_backward_launches(const lh_config* cfg) {
+  if (check(cfg) != LH_OK) return -1;
+  return 1 + 2 + 1;  // scatter_bwd, attention dK/dV and dQ, gather_bwd
+}
+
+}  // extern "C"

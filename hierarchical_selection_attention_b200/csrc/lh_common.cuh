@@ -1,0 +1,90 @@
+// Internal helpers shared by the Lighthouse kernels: derived sizes, bf16
+// packing, the device status word and bounded waits.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lighthouse.h"
+
+#define LH_MAX_LEVELS 8
+
+// Sizes derived once on the host from an lh_config and passed by value.
+struct LhDims {
+  int B, H, d, L, p;
+  int64_t N;
+  int64_t S;                      // gathered length (Eq. 8)
+  int64_t P;                      // pyramid entries per (b, h)
+  int64_t n_cand;                 // entries of levels 0..L-2
+  int64_t n_sel;                  // (L-1) p k
+  int64_t lvl_size[LH_MAX_LEVELS];   // N / p^l
+  int64_t lvl_off[LH_MAX_LEVELS];    // flat offset of level l
+  int64_t lvl_span[LH_MAX_LEVELS];   // p^l
+  int64_t pool_row[LH_MAX_LEVELS];   // first pooled row of level l (l >= 1), per batch row
+  int64_t pooled_rows;               // sum_{l>=1} N / p^l
+  float scale;
+  int* status;                       // device status word [code, detail]
+};
+
+// Device status word: first error wins.  Codes are lh_status values; the
+// detail word says which wait or check failed.
+__device__ __forceinline__ void lh_report(int* status, int code, int detail) {
+  if (atomicCAS(status, 0, code) == 0) atomicExch(status + 1, detail);
+}
+
+// Level of a flat pyramid index (levels are few; a linear scan is cheapest).
+__device__ __forceinline__ int lh_level_of(const LhDims& D, int64_t f) {
+  int l = 0;
+#pragma unroll 1
+  for (int j = 1; j < D.L; ++j)
+    if (f >= D.lvl_off[j]) l = j;
+  return l;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
+  float2 r;
+  r.x = __uint_as_float(u << 16);
+  r.y = __uint_as_float(u & 0xffff0000u);
+  return r;
+}
+
+// Host side launchers (one per kernel family), all enqueue on `st`.
+cudaError_t lh_launch_pyramid(const LhDims& D, const lh_bf16* q, const lh_bf16* k,
+                              const lh_bf16* v, lh_bf16* q_lv, lh_bf16* k_lv, lh_bf16* v_lv,
+                              float* qk, float* kq, cudaStream_t st);
+size_t lh_select_ws_bytes(const LhDims& D);
+cudaError_t lh_launch_select(const LhDims& D, const float* qk, const float* kq,
+                             int32_t* sel_idx, int32_t* slot_map, void* ws, cudaStream_t st,
+                             int* launches);
+cudaError_t lh_launch_gather(const LhDims& D, const lh_bf16* q, const lh_bf16* k,
+                             const lh_bf16* v, const lh_bf16* q_lv, const lh_bf16* k_lv,
+                             const lh_bf16* v_lv, const int32_t* sel_idx, lh_bf16* qg,
+                             lh_bf16* kg, lh_bf16* vg, cudaStream_t st);
+cudaError_t lh_launch_scatter(const LhDims& D, const lh_bf16* og, const int32_t* slot_map,
+                              lh_bf16* o, cudaStream_t st);
+size_t lh_scatter_atomic_ws_bytes(const LhDims& D);
+cudaError_t lh_launch_scatter_atomic(const LhDims& D, const lh_bf16* og,
+                                     const int32_t* slot_map, lh_bf16* o, void* ws,
+                                     cudaStream_t st, int* launches);
+cudaError_t lh_launch_scatter_bwd(const LhDims& D, const lh_bf16* dout, const lh_bf16* og,
+                                  const int32_t* sel_idx, lh_bf16* dog, float* delta,
+                                  cudaStream_t st);
+cudaError_t lh_launch_gather_bwd(const LhDims& D, const lh_bf16* dqg, const lh_bf16* dkg,
+                                 const lh_bf16* dvg, const int32_t* slot_map, lh_bf16* dq,
+                                 lh_bf16* dk, lh_bf16* dv, cudaStream_t st);
+cudaError_t lh_launch_attn_fwd(int BH, int64_t S, int d, float scale, const lh_bf16* qg,
+                               const lh_bf16* kg, const lh_bf16* vg, lh_bf16* og, float* lse,
+                               int* status, cudaStream_t st);
+cudaError_t lh_launch_attn_delta(int BH, int64_t S, int d, const lh_bf16* og,
+                                 const lh_bf16* dog, float* delta, cudaStream_t st);
+cudaError_t lh_launch_attn_bwd(int BH, int64_t S, int d, float scale, const lh_bf16* qg,
+                               const lh_bf16* kg, const lh_bf16* vg, const lh_bf16* dog,
+                               const float* lse, const float* delta, lh_bf16* dqg,
+                               lh_bf16* dkg, lh_bf16* dvg, int* status, cudaStream_t st,
+                               int* launches);

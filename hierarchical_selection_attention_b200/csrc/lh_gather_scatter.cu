@@ -1,0 +1,316 @@
+// Data movement around the attention of Lighthouse Attention ("Long Context
+// Pre-Training with Lighthouse Attention", Sec. 3.5 gather, Sec. 3.6
+// scatter-back) and the adjoints of both (Sec. 3.2: gradients flow through
+// the scatter, the attention and the gather).
+//
+// All kernels are HBM-bound.  One thread moves one 16-byte vector (8 bf16
+// features) of one row; consecutive threads take consecutive vectors of a
+// row, so warp accesses are whole 256-byte (d = 128) or 128-byte (d = 64)
+// rows, and index loads are shared by the d/8 threads of a row.  Sums run in
+// fp32 in a fixed order (ascending level, ascending token) and are rounded
+// once to bf16, so every output is deterministic.
+#include "lh_common.cuh"
+
+namespace {
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ void acc8(float* a, const uint4& u, float s = 1.f) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = unpack_bf16x2(w[e]);
+    a[2 * e] = fmaf(f.x, s, a[2 * e]);
+    a[2 * e + 1] = fmaf(f.y, s, a[2 * e + 1]);
+  }
+}
+
+__device__ __forceinline__ uint4 pack8(const float* a) {
+  uint4 u;
+  u.x = pack_bf16x2(a[0], a[1]);
+  u.y = pack_bf16x2(a[2], a[3]);
+  u.z = pack_bf16x2(a[4], a[5]);
+  u.w = pack_bf16x2(a[6], a[7]);
+  return u;
+}
+
+// Vector index of row (b, i, h) of level l in the pyramid: level 0 is the
+// input tensor, level l >= 1 lives in the pooled buffer.
+__device__ __forceinline__ const uint4* level_row(const LhDims& D, const uint4* x0,
+                                                  const uint4* xl, int l, int b, int64_t i,
+                                                  int h, int V) {
+  if (l == 0) return x0 + (((int64_t)b * D.N + i) * D.H + h) * V;
+  return xl + (((int64_t)D.B * D.pool_row[l] + (int64_t)b * D.lvl_size[l] + i) * D.H + h) * V;
+}
+
+// (iii) gather: thread = (b, h, slot m, vector cv).
+__global__ void __launch_bounds__(kThreads) k_gather(LhDims D, const uint4* __restrict__ q,
+                                                     const uint4* __restrict__ k,
+                                                     const uint4* __restrict__ v,
+                                                     const uint4* __restrict__ q_lv,
+                                                     const uint4* __restrict__ k_lv,
+                                                     const uint4* __restrict__ v_lv,
+                                                     const int32_t* __restrict__ sel_idx,
+                                                     uint4* __restrict__ qg, uint4* __restrict__ kg,
+                                                     uint4* __restrict__ vg) {
+  const int V = D.d >> 3;
+  const int64_t item = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t total = (int64_t)D.B * D.H * D.S * V;
+  if (item >= total) return;
+  const int cv = (int)(item % V);
+  const int64_t row = item / V;  // (bh, m)
+  const int64_t bh = row / D.S;
+  const int b = (int)(bh / D.H), h = (int)(bh % D.H);
+  const int64_t f = __ldg(sel_idx + row);
+  if (f < 0 || f >= D.P) {
+    lh_report(D.status, LH_ERR_DEVICE_BOUNDS, 200);
+    return;
+  }
+  const int l = lh_level_of(D, f);
+  const int64_t i = f - D.lvl_off[l];
+  const int64_t o = row * V + cv;
+  qg[o] = __ldg(level_row(D, q, q_lv, l, b, i, h, V) + cv);
+  kg[o] = __ldg(level_row(D, k, k_lv, l, b, i, h, V) + cv);
+  vg[o] = __ldg(level_row(D, v, v_lv, l, b, i, h, V) + cv);
+}
+
+// (iv) scatter-back, gather side: thread = (b, t, h, vector cv); the entry of
+// level l that reaches t is i = floor((t+1)/p^l) - 1.
+__global__ void __launch_bounds__(kThreads) k_scatter(LhDims D, const uint4* __restrict__ og,
+                                                      const int32_t* __restrict__ slot_map,
+                                                      uint4* __restrict__ o) {
+  const int V = D.d >> 3;
+  const int64_t item = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t total = (int64_t)D.B * D.N * D.H * V;
+  if (item >= total) return;
+  const int cv = (int)(item % V);
+  const int64_t r = item / V;  // (b, t, h)
+  const int h = (int)(r % D.H);
+  const int64_t bt = r / D.H;
+  const int64_t t = bt % D.N;
+  const int b = (int)(bt / D.N);
+  const int64_t bh = (int64_t)b * D.H + h;
+  const int32_t* sm = slot_map + bh * D.P;
+  float a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  const uint32_t t1 = (uint32_t)(t + 1);
+  for (int l = 0; l < D.L; ++l) {
+    const uint32_t j = t1 / (uint32_t)D.lvl_span[l];
+    if (j == 0) break;
+    const int slot = __ldg(sm + D.lvl_off[l] + j - 1);
+    if (slot < 0) continue;
+    acc8(a, __ldg(og + (bh * D.S + slot) * V + cv));
+  }
+  o[item] = pack8(a);
+}
+
+// (iv) in fixed-point integer atomics: every selected entry adds its output,
+// scaled by 2^32 and rounded to an integer, into the 64-bit accumulators of
+// its shifted range; integer addition is associative, so the sums do not
+// depend on the order the atomics land in.  Thread = (b, h, entry f, pair of
+// features); unselected entries leave at once.
+__global__ void __launch_bounds__(kThreads) k_scatter_push(LhDims D, const uint32_t* __restrict__ og,
+                                                           const int32_t* __restrict__ slot_map,
+                                                           unsigned long long* __restrict__ acc) {
+  const int Vp = D.d >> 1;  // bf16 pairs per row
+  const int64_t item = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t total = (int64_t)D.B * D.H * D.P * Vp;
+  if (item >= total) return;
+  const int c2 = (int)(item % Vp);
+  const int64_t ent = item / Vp;        // (bh, f)
+  const int64_t bh = ent / D.P;
+  const int64_t f = ent % D.P;
+  const int slot = __ldg(slot_map + ent);
+  if (slot < 0) return;
+  const int b = (int)(bh / D.H), h = (int)(bh % D.H);
+  const int l = lh_level_of(D, f);
+  const int64_t i = f - D.lvl_off[l];
+  const int64_t span = D.lvl_span[l];
+  const int64_t start = (i + 1) * span - 1;
+  const int64_t stop = min(start + span, D.N);
+  const float2 x = unpack_bf16x2(__ldg(og + (bh * D.S + slot) * Vp + c2));
+  const long long ix = __double2ll_rn((double)x.x * 4294967296.0);
+  const long long iy = __double2ll_rn((double)x.y * 4294967296.0);
+  for (int64_t t = start; t < stop; ++t) {
+    unsigned long long* dst = acc + (((int64_t)b * D.N + t) * D.H + h) * D.d + 2 * c2;
+    atomicAdd(dst, (unsigned long long)ix);
+    atomicAdd(dst + 1, (unsigned long long)iy);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads) k_scatter_fix2bf16(int64_t n,
+                                                               const long long* __restrict__ acc,
+                                                               uint32_t* __restrict__ o) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float a = (float)((double)acc[2 * i] * (1.0 / 4294967296.0));
+  const float b = (float)((double)acc[2 * i + 1] * (1.0 / 4294967296.0));
+  o[i] = pack_bf16x2(a, b);
+}
+
+// Adjoint of the scatter, fused with D = rowsum(dog * og): thread = (b, h,
+// slot m, vector cv); it sums dO over the shifted range of the slot's entry.
+__global__ void __launch_bounds__(kThreads) k_scatter_bwd(LhDims D, const uint4* __restrict__ dout,
+                                                          const uint4* __restrict__ og,
+                                                          const int32_t* __restrict__ sel_idx,
+                                                          uint4* __restrict__ dog,
+                                                          float* __restrict__ delta) {
+  const int V = D.d >> 3;
+  const int64_t item = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t total = (int64_t)D.B * D.H * D.S * V;
+  const unsigned live = __ballot_sync(0xffffffffu, item < total);
+  if (item >= total) return;
+  const int cv = (int)(item % V);
+  const int64_t row = item / V;
+  const int64_t bh = row / D.S;
+  const int b = (int)(bh / D.H), h = (int)(bh % D.H);
+  const int64_t f = __ldg(sel_idx + row);
+  const int l = lh_level_of(D, f);
+  const int64_t i = f - D.lvl_off[l];
+  const int64_t span = D.lvl_span[l];
+  const int64_t start = (i + 1) * span - 1;
+  const int64_t stop = min(start + span, D.N);
+  const int64_t HV = (int64_t)D.H * V;
+  const uint4* src = dout + ((int64_t)b * D.N * D.H + h) * V + cv;
+  float a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  int64_t t = start;
+  for (; t + 4 <= stop; t += 4) {
+    const uint4 u0 = __ldg(src + t * HV), u1 = __ldg(src + (t + 1) * HV);
+    const uint4 u2 = __ldg(src + (t + 2) * HV), u3 = __ldg(src + (t + 3) * HV);
+    acc8(a, u0); acc8(a, u1); acc8(a, u2); acc8(a, u3);
+  }
+  for (; t < stop; ++t) acc8(a, __ldg(src + t * HV));
+  const uint4 packed = pack8(a);
+  dog[item] = packed;
+  // D from the stored (rounded) values, as the attention backward sees them
+  float rd[8] = {0, 0, 0, 0, 0, 0, 0, 0}, ro[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  acc8(rd, packed);
+  acc8(ro, __ldg(og + item));
+  float s = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) s = fmaf(rd[e], ro[e], s);
+  for (int o = V >> 1; o > 0; o >>= 1) s += __shfl_xor_sync(live, s, o);
+  if (cv == 0) delta[row] = s;
+}
+
+// D = rowsum(dog * og) for the standalone attention backward.
+__global__ void __launch_bounds__(kThreads) k_attn_delta(int64_t rows, int V,
+                                                         const uint4* __restrict__ og,
+                                                         const uint4* __restrict__ dog,
+                                                         float* __restrict__ delta) {
+  const int64_t item = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const unsigned live = __ballot_sync(0xffffffffu, item < rows * V);
+  if (item >= rows * V) return;
+  float rd[8] = {0, 0, 0, 0, 0, 0, 0, 0}, ro[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  acc8(rd, __ldg(dog + item));
+  acc8(ro, __ldg(og + item));
+  float s = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) s = fmaf(rd[e], ro[e], s);
+  for (int o = V >> 1; o > 0; o >>= 1) s += __shfl_xor_sync(live, s, o);
+  if (item % V == 0) delta[item / V] = s;
+}
+
+// Adjoint of gather + mean pooling: thread = (b, t, h, vector cv); the level-l
+// entry whose (unshifted) window holds t is i = floor(t / p^l).
+__global__ void __launch_bounds__(kThreads) k_gather_bwd(LhDims D, const uint4* __restrict__ dqg,
+                                                         const uint4* __restrict__ dkg,
+                                                         const uint4* __restrict__ dvg,
+                                                         const int32_t* __restrict__ slot_map,
+                                                         uint4* __restrict__ dq, uint4* __restrict__ dk,
+                                                         uint4* __restrict__ dv) {
+  const int V = D.d >> 3;
+  const int64_t item = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t total = (int64_t)D.B * D.N * D.H * V;
+  if (item >= total) return;
+  const int cv = (int)(item % V);
+  const int64_t r = item / V;
+  const int h = (int)(r % D.H);
+  const int64_t bt = r / D.H;
+  const int64_t t = bt % D.N;
+  const int b = (int)(bt / D.N);
+  const int64_t bh = (int64_t)b * D.H + h;
+  const int32_t* sm = slot_map + bh * D.P;
+  float aq[8] = {0, 0, 0, 0, 0, 0, 0, 0}, ak[8] = {0, 0, 0, 0, 0, 0, 0, 0},
+        av[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (int l = 0; l < D.L; ++l) {
+    const uint32_t i = (uint32_t)t / (uint32_t)D.lvl_span[l];
+    const int slot = __ldg(sm + D.lvl_off[l] + i);
+    if (slot < 0) continue;
+    const float w = 1.f / (float)D.lvl_span[l];
+    const int64_t s = (bh * D.S + slot) * V + cv;
+    acc8(aq, __ldg(dqg + s), w);
+    acc8(ak, __ldg(dkg + s), w);
+    acc8(av, __ldg(dvg + s), w);
+  }
+  dq[item] = pack8(aq);
+  dk[item] = pack8(ak);
+  dv[item] = pack8(av);
+}
+
+inline unsigned nblocks(int64_t n) { return (unsigned)((n + kThreads - 1) / kThreads); }
+
+}  // namespace
+
+cudaError_t lh_launch_gather(const LhDims& D, const lh_bf16* q, const lh_bf16* k,
+                             const lh_bf16* v, const lh_bf16* q_lv, const lh_bf16* k_lv,
+                             const lh_bf16* v_lv, const int32_t* sel_idx, lh_bf16* qg,
+                             lh_bf16* kg, lh_bf16* vg, cudaStream_t st) {
+  const int64_t n = (int64_t)D.B * D.H * D.S * (D.d >> 3);
+  k_gather<<<nblocks(n), kThreads, 0, st>>>(
+      D, (const uint4*)q, (const uint4*)k, (const uint4*)v, (const uint4*)q_lv,
+      (const uint4*)k_lv, (const uint4*)v_lv, sel_idx, (uint4*)qg, (uint4*)kg, (uint4*)vg);
+  return cudaGetLastError();
+}
+
+cudaError_t lh_launch_scatter(const LhDims& D, const lh_bf16* og, const int32_t* slot_map,
+                              lh_bf16* o, cudaStream_t st) {
+  const int64_t n = (int64_t)D.B * D.N * D.H * (D.d >> 3);
+  k_scatter<<<nblocks(n), kThreads, 0, st>>>(D, (const uint4*)og, slot_map, (uint4*)o);
+  return cudaGetLastError();
+}
+
+size_t lh_scatter_atomic_ws_bytes(const LhDims& D) {
+  return (size_t)D.B * D.N * D.H * D.d * sizeof(long long);
+}
+
+cudaError_t lh_launch_scatter_atomic(const LhDims& D, const lh_bf16* og,
+                                     const int32_t* slot_map, lh_bf16* o, void* ws,
+                                     cudaStream_t st, int* launches) {
+  const int64_t elems = (int64_t)D.B * D.N * D.H * D.d;
+  cudaError_t e = cudaMemsetAsync(ws, 0, (size_t)elems * sizeof(long long), st);
+  if (e != cudaSuccess) return e;
+  const int64_t n = (int64_t)D.B * D.H * D.P * (D.d >> 1);
+  k_scatter_push<<<nblocks(n), kThreads, 0, st>>>(D, (const uint32_t*)og, slot_map,
+                                                  (unsigned long long*)ws);
+  k_scatter_fix2bf16<<<nblocks(elems / 2), kThreads, 0, st>>>(elems / 2, (const long long*)ws,
+                                                             (uint32_t*)o);
+  if (launches) *launches = 2;
+  return cudaGetLastError();
+}
+
+cudaError_t lh_launch_scatter_bwd(const LhDims& D, const lh_bf16* dout, const lh_bf16* og,
+                                  const int32_t* sel_idx, lh_bf16* dog, float* delta,
+                                  cudaStream_t st) {
+  const int64_t n = (int64_t)D.B * D.H * D.S * (D.d >> 3);
+  k_scatter_bwd<<<nblocks(n), kThreads, 0, st>>>(D, (const uint4*)dout, (const uint4*)og, sel_idx,
+                                                 (uint4*)dog, delta);
+  return cudaGetLastError();
+}
+
+cudaError_t lh_launch_attn_delta(int BH, int64_t S, int d, const lh_bf16* og,
+                                 const lh_bf16* dog, float* delta, cudaStream_t st) {
+  const int64_t rows = (int64_t)BH * S;
+  k_attn_delta<<<nblocks(rows * (d >> 3)), kThreads, 0, st>>>(rows, d >> 3, (const uint4*)og,
+                                                             (const uint4*)dog, delta);
+  return cudaGetLastError();
+}
+
+cudaError_t lh_launch_gather_bwd(const LhDims& D, const lh_bf16* dqg, const lh_bf16* dkg,
+                                 const lh_bf16* dvg, const int32_t* slot_map, lh_bf16* dq,
+                                 lh_bf16* dk, lh_bf16* dv, cudaStream_t st) {
+  const int64_t n = (int64_t)D.B * D.N * D.H * (D.d >> 3);
+  k_gather_bwd<<<nblocks(n), kThreads, 0, st>>>(D, (const uint4*)dqg, (const uint4*)dkg,
+                                                (const uint4*)dvg, slot_map, (uint4*)dq,
+                                                (uint4*)dk, (uint4*)dv);
+  return cudaGetLastError();
+}

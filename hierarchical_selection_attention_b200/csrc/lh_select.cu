@@ -1,0 +1,300 @@
+// Stage (ii) selection and the topological order of stage (iii)
+// ("Long Context Pre-Training with Lighthouse Attention", Sec. 3.4 and 3.5).
+//
+// Joint top-k.  Every finer-level entry f (levels 0..L-2) gets the unique
+// 64-bit key
+//      key(f) = bits(max(QK_f, KQ_f)) << 32  |  (2^32 - 1 - f)
+// (scores are >= 0, so their fp32 bit patterns order like the values, and the
+// low word makes the lower flat index win a tie).  Taking distinct entries
+// from the QK and KQ streams merged by score is the same as taking the n_sel
+// largest keys, because an entry first shows up at the larger of its two
+// scores.  The n_sel-th largest key is found by radix selection, 11 bits per
+// pass from the top: a histogram pass counts the digits of the keys that
+// still match the prefix found so far, and a one-block pass picks the digit
+// that holds the n_sel-th key.  Once every key left in that digit is needed,
+// the threshold is final and later passes return at once.  Then
+// selected(f) <=> key(f) >= threshold: integer work only, so the selected
+// set is bit-exact and the same on every run.
+//
+// Order.  Entries are sorted by the last base token they summarise,
+// e = (i+1) p^l - 1, and by level.  Walking the base tokens t in order and,
+// for each, the levels whose entries end at t ((t+1) mod p^l == 0) in
+// ascending order lists the selected entries in exactly that order, so slots
+// come from a prefix sum over t of the number of selected entries ending at
+// t: a counting pass per block of tokens, a scan over blocks, and an emit
+// pass that writes sel_idx (slot -> entry) and slot_map (entry -> slot or -1).
+#include <cub/block/block_reduce.cuh>
+#include <cub/block/block_scan.cuh>
+
+#include "lh_common.cuh"
+
+namespace {
+
+constexpr int kPasses = 6;
+constexpr int kBins = 2048;
+__constant__ int c_shift[kPasses] = {53, 42, 31, 20, 9, 0};
+__constant__ int c_width[kPasses] = {11, 11, 11, 11, 11, 9};
+
+struct SelState {
+  unsigned long long prefix;  // digits fixed so far (lower bits zero)
+  long long need;             // keys still to take among those matching prefix
+  int done;                   // threshold final
+  int pad;
+};
+
+constexpr int kOrderThreads = 256;
+constexpr int kOrderItems = 4;                        // tokens per thread
+constexpr int kOrderTile = kOrderThreads * kOrderItems;
+
+__device__ __forceinline__ unsigned long long entry_key(const float* qk, const float* kq,
+                                                        int64_t f) {
+  const float r = fmaxf(__ldg(qk + f), __ldg(kq + f));
+  return ((unsigned long long)__float_as_uint(r) << 32) |
+         (unsigned long long)(0xffffffffu - (uint32_t)f);
+}
+
+__global__ void __launch_bounds__(256) k_sel_hist(LhDims D, const float* __restrict__ qk,
+                                                  const float* __restrict__ kq,
+                                                  unsigned* __restrict__ hist,
+                                                  const SelState* __restrict__ state, int pass) {
+  const int64_t bh = blockIdx.y;
+  unsigned long long prefix = 0;
+  if (pass > 0) {
+    const SelState s = state[bh];
+    if (s.done) return;
+    prefix = s.prefix;
+  }
+  __shared__ unsigned h[kBins];
+  for (int i = threadIdx.x; i < kBins; i += blockDim.x) h[i] = 0;
+  __syncthreads();
+  const int shift = c_shift[pass];
+  const int hi = shift + c_width[pass];
+  const unsigned mask = (1u << c_width[pass]) - 1u;
+  const float* q = qk + bh * D.P;
+  const float* k = kq + bh * D.P;
+  const int64_t per_block = (D.n_cand + gridDim.x - 1) / gridDim.x;
+  const int64_t lo = (int64_t)blockIdx.x * per_block;
+  const int64_t end = min(lo + per_block, D.n_cand);
+  const int64_t span = end > lo ? end - lo : 0;
+  const int64_t rounds = (span + blockDim.x - 1) / blockDim.x;
+  for (int64_t r = 0; r < rounds; ++r) {
+    const int64_t f = lo + r * blockDim.x + threadIdx.x;
+    bool in = f < end;
+    unsigned digit = 0;
+    if (in) {
+      const unsigned long long key = entry_key(q, k, f);
+      in = (hi >= 64) || ((key >> hi) == (prefix >> hi));
+      digit = (unsigned)(key >> shift) & mask;
+    }
+    // warp-aggregated increment: one shared atomic per distinct digit
+    const unsigned act = __ballot_sync(0xffffffffu, in);
+    if (in) {
+      const unsigned peers = __match_any_sync(act, digit);
+      if ((threadIdx.x & 31) == (unsigned)(__ffs(peers) - 1)) atomicAdd(&h[digit], __popc(peers));
+    }
+  }
+  __syncthreads();
+  unsigned* g = hist + (bh * kPasses + pass) * kBins;
+  for (int i = threadIdx.x; i < kBins; i += blockDim.x)
+    if (h[i]) atomicAdd(&g[i], h[i]);
+}
+
+// One block of 256 threads per (b, h); thread t owns digits 2047-8t .. 2040-8t.
+__global__ void __launch_bounds__(256) k_sel_find(LhDims D, const unsigned* __restrict__ hist,
+                                                  SelState* __restrict__ state, int pass) {
+  const int64_t bh = blockIdx.x;
+  SelState s;
+  if (pass == 0) {
+    s.prefix = 0;
+    s.need = D.n_sel;
+    s.done = D.n_sel == 0;
+    s.pad = 0;
+    if (s.done) s.prefix = ~0ull;  // nothing is selected
+  } else {
+    s = state[bh];
+  }
+  __syncthreads();
+  if (s.done) {
+    if (pass == 0 && threadIdx.x == 0) state[bh] = s;
+    return;
+  }
+  const unsigned* g = hist + (bh * kPasses + pass) * kBins;
+  unsigned c[8];
+  long long mine = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    c[i] = g[kBins - 1 - (threadIdx.x * 8 + i)];
+    mine += c[i];
+  }
+  typedef cub::BlockScan<long long, 256> Scan;
+  __shared__ typename Scan::TempStorage tmp;
+  long long before;
+  Scan(tmp).ExclusiveSum(mine, before);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (before < s.need && s.need <= before + (long long)c[i]) {
+      const unsigned digit = kBins - 1 - (threadIdx.x * 8 + i);
+      SelState o;
+      o.prefix = s.prefix | ((unsigned long long)digit << c_shift[pass]);
+      o.need = s.need - before;
+      o.done = (o.need == (long long)c[i]) ? 1 : 0;
+      o.pad = 0;
+      state[bh] = o;
+      if (!o.done && pass == kPasses - 1) lh_report(D.status, LH_ERR_DEVICE_BOUNDS, 100);
+    }
+    before += c[i];
+  }
+}
+
+__device__ __forceinline__ bool selected_entry(const LhDims& D, const float* q, const float* k,
+                                               unsigned long long thr, int l, int64_t f) {
+  return (l == D.L - 1) || (entry_key(q, k, f) >= thr);
+}
+
+// Number of selected entries that end on token t.
+__device__ __forceinline__ int count_at(const LhDims& D, const float* q, const float* k,
+                                        unsigned long long thr, int64_t t) {
+  int n = 0;
+  const uint32_t t1 = (uint32_t)(t + 1);  // N < 2^31
+  for (int l = 0; l < D.L; ++l) {
+    const uint32_t span = (uint32_t)D.lvl_span[l];
+    if (t1 % span) break;  // spans are nested: no coarser level ends here either
+    n += selected_entry(D, q, k, thr, l, D.lvl_off[l] + t1 / span - 1);
+  }
+  return n;
+}
+
+__global__ void __launch_bounds__(kOrderThreads) k_order_count(LhDims D, const float* __restrict__ qk,
+                                                              const float* __restrict__ kq,
+                                                              const SelState* __restrict__ state,
+                                                              int* __restrict__ blk_cnt, int nblk) {
+  const int64_t bh = blockIdx.y;
+  const unsigned long long thr = state[bh].prefix;
+  const float* q = qk + bh * D.P;
+  const float* k = kq + bh * D.P;
+  const int64_t t0 = (int64_t)blockIdx.x * kOrderTile;
+  int n = 0;
+  for (int i = 0; i < kOrderItems; ++i) {
+    const int64_t t = t0 + (int64_t)i * kOrderThreads + threadIdx.x;
+    if (t < D.N) n += count_at(D, q, k, thr, t);
+  }
+  typedef cub::BlockReduce<int, kOrderThreads> Red;
+  __shared__ typename Red::TempStorage tmp;
+  const int tot = Red(tmp).Sum(n);
+  if (threadIdx.x == 0) blk_cnt[bh * nblk + blockIdx.x] = tot;
+}
+
+// One block per (b, h): exclusive scan of the block counts, in place.
+__global__ void __launch_bounds__(1024) k_order_scan(LhDims D, int* __restrict__ blk_cnt, int nblk) {
+  const int64_t bh = blockIdx.x;
+  int* c = blk_cnt + bh * nblk;
+  typedef cub::BlockScan<int, 1024> Scan;
+  __shared__ typename Scan::TempStorage tmp;
+  __shared__ int carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < nblk; base += 1024) {
+    const int i = base + threadIdx.x;
+    const int x = i < nblk ? c[i] : 0;
+    int ex, agg;
+    Scan(tmp).ExclusiveSum(x, ex, agg);
+    if (i < nblk) c[i] = carry + ex;
+    __syncthreads();
+    if (threadIdx.x == 0) carry += agg;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0 && carry != D.S) lh_report(D.status, LH_ERR_DEVICE_BOUNDS, 101);
+}
+
+__global__ void __launch_bounds__(kOrderThreads) k_order_emit(LhDims D, const float* __restrict__ qk,
+                                                             const float* __restrict__ kq,
+                                                             const SelState* __restrict__ state,
+                                                             const int* __restrict__ blk_off, int nblk,
+                                                             int32_t* __restrict__ sel_idx,
+                                                             int32_t* __restrict__ slot_map) {
+  const int64_t bh = blockIdx.y;
+  const unsigned long long thr = state[bh].prefix;
+  const float* q = qk + bh * D.P;
+  const float* k = kq + bh * D.P;
+  // each thread owns kOrderItems consecutive tokens so the scan order is t order
+  const int64_t t0 = (int64_t)blockIdx.x * kOrderTile + (int64_t)threadIdx.x * kOrderItems;
+  int n = 0;
+  for (int i = 0; i < kOrderItems; ++i) {
+    const int64_t t = t0 + i;
+    if (t < D.N) n += count_at(D, q, k, thr, t);
+  }
+  typedef cub::BlockScan<int, kOrderThreads> Scan;
+  __shared__ typename Scan::TempStorage tmp;
+  int ex;
+  Scan(tmp).ExclusiveSum(n, ex);
+  int slot = blk_off[bh * nblk + blockIdx.x] + ex;
+  int32_t* si = sel_idx + bh * D.S;
+  int32_t* sm = slot_map + bh * D.P;
+  for (int i = 0; i < kOrderItems; ++i) {
+    const int64_t t = t0 + i;
+    if (t >= D.N) break;
+    const uint32_t t1 = (uint32_t)(t + 1);
+    for (int l = 0; l < D.L; ++l) {
+      const uint32_t span = (uint32_t)D.lvl_span[l];
+      if (t1 % span) break;
+      const int64_t f = D.lvl_off[l] + t1 / span - 1;
+      if (selected_entry(D, q, k, thr, l, f)) {
+        if (slot < D.S) si[slot] = (int32_t)f;
+        else lh_report(D.status, LH_ERR_DEVICE_BOUNDS, 102);
+        sm[f] = slot++;
+      } else {
+        sm[f] = -1;
+      }
+    }
+  }
+}
+
+inline int64_t order_blocks(const LhDims& D) { return (D.N + kOrderTile - 1) / kOrderTile; }
+
+}  // namespace
+
+size_t lh_select_ws_bytes(const LhDims& D) {
+  const int64_t BH = (int64_t)D.B * D.H;
+  size_t b = 0;
+  b += (size_t)BH * kPasses * kBins * sizeof(unsigned);
+  b += (size_t)BH * sizeof(SelState);
+  b = (b + 255) & ~(size_t)255;
+  b += (size_t)BH * order_blocks(D) * sizeof(int);
+  return (b + 255) & ~(size_t)255;
+}
+
+cudaError_t lh_launch_select(const LhDims& D, const float* qk, const float* kq,
+                             int32_t* sel_idx, int32_t* slot_map, void* ws, cudaStream_t st,
+                             int* launches) {
+  const int64_t BH = (int64_t)D.B * D.H;
+  unsigned* hist = reinterpret_cast<unsigned*>(ws);
+  SelState* state = reinterpret_cast<SelState*>(hist + BH * kPasses * kBins);
+  size_t off = (size_t)BH * kPasses * kBins * sizeof(unsigned) + (size_t)BH * sizeof(SelState);
+  off = (off + 255) & ~(size_t)255;
+  int* blk = reinterpret_cast<int*>(reinterpret_cast<char*>(ws) + off);
+  const int nblk = (int)order_blocks(D);
+  int n = 0;
+  cudaError_t e = cudaMemsetAsync(hist, 0, (size_t)BH * kPasses * kBins * sizeof(unsigned), st);
+  if (e != cudaSuccess) return e;
+  if (D.n_cand > 0) {
+    // ~8 candidates per thread per block keeps every SM busy on one head too
+    int64_t per = (D.n_cand + 148 * 4 - 1) / (148 * 4);
+    per = per < 2048 ? 2048 : per;
+    const unsigned gx = (unsigned)((D.n_cand + per - 1) / per);
+    for (int pass = 0; pass < kPasses; ++pass) {
+      k_sel_hist<<<dim3(gx, (unsigned)BH), 256, 0, st>>>(D, qk, kq, hist, state, pass);
+      k_sel_find<<<(unsigned)BH, 256, 0, st>>>(D, hist, state, pass);
+      n += 2;
+    }
+  } else {
+    k_sel_find<<<(unsigned)BH, 256, 0, st>>>(D, hist, state, 0);
+    n += 1;
+  }
+  k_order_count<<<dim3(nblk, (unsigned)BH), kOrderThreads, 0, st>>>(D, qk, kq, state, blk, nblk);
+  k_order_scan<<<(unsigned)BH, 1024, 0, st>>>(D, blk, nblk);
+  k_order_emit<<<dim3(nblk, (unsigned)BH), kOrderThreads, 0, st>>>(D, qk, kq, state, blk, nblk,
+                                                                   sel_idx, slot_map);
+  n += 3;
+  if (launches) *launches = n;
+  return cudaGetLastError();
+}

@@ -1,0 +1,293 @@
+"""ctypes binding of liblighthouse.so, the C ABI in include/lighthouse.h.
+
+Argument marshalling only: every function below checks that the tensors
+have the dtype, size and device the C call expects, passes their device
+pointers and torch's current CUDA stream, and raises LighthouseError if the
+library returns an error.  All work runs in the library's CUDA kernels.
+The library must be built (``python -m hierarchical_selection_attention_b200.build``);
+importing this module without it raises at once, there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblighthouse.so")
+
+LH_OK = 0
+_STATUS = {0: "LH_OK", 1: "LH_ERR_INVALID_ARGUMENT", 2: "LH_ERR_UNSUPPORTED",
+           3: "LH_ERR_WORKSPACE", 4: "LH_ERR_CUDA", 5: "LH_ERR_DEVICE_TIMEOUT",
+           6: "LH_ERR_DEVICE_BOUNDS"}
+
+
+class LighthouseError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {_STATUS.get(code, code)} ({_lib.lh_status_string(code).decode()})")
+
+
+class lh_config(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int64), ("N", ctypes.c_int64), ("H", ctypes.c_int64),
+                ("d", ctypes.c_int64), ("L", ctypes.c_int64), ("p", ctypes.c_int64),
+                ("k", ctypes.c_int64), ("scale", ctypes.c_float),
+                ("scatter_mode", ctypes.c_int32), ("select_mode", ctypes.c_int32)]
+
+    def as_dict(self):
+        return {f: getattr(self, f) for f, _ in self._fields_}
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m hierarchical_selection_attention_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I64, I32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+    C = ctypes.POINTER(lh_config)
+    sig = {
+        "lh_config_check": (I32, [C]),
+        "lh_subseq_len": (I64, [C]),
+        "lh_total_entries": (I64, [C]),
+        "lh_pooled_rows": (I64, [C]),
+        "lh_workspace_bytes": (I32, [C, ctypes.POINTER(SZ), ctypes.POINTER(SZ), ctypes.POINTER(SZ)]),
+        "lh_saved_offsets": (I32, [C, ctypes.POINTER(SZ)]),
+        "lh_pyramid": (I32, [C, P, P, P, P, P, P, P, P, P]),
+        "lh_score_topk": (I32, [C, P, P, P, P, P, SZ, P]),
+        "lh_gather": (I32, [C, P, P, P, P, P, P, P, P, P, P, P]),
+        "lh_attn_fwd": (I32, [C, P, P, P, P, P, P]),
+        "lh_attn_bwd": (I32, [C, P, P, P, P, P, P, P, P, P, P, SZ, P]),
+        "lh_scatter": (I32, [C, P, P, P, P, SZ, P]),
+        "lh_scatter_bwd": (I32, [C, P, P, P, P, P, P]),
+        "lh_gather_bwd": (I32, [C, P, P, P, P, P, P, P, P]),
+        "lh_forward": (I32, [C, P, P, P, P, P, SZ, P, SZ, P]),
+        "lh_backward": (I32, [C, P, SZ, P, P, P, P, P, SZ, P]),
+        "lh_get_device_status": (I32, [P, ctypes.POINTER(I32)]),
+        "lh_status_string": (ctypes.c_char_p, [I32]),
+        "lh_forward_launches": (I32, [C]),
+        "lh_backward_launches": (I32, [C]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype, fn.argtypes = res, args
+    return lib
+
+
+_lib = _load()
+EXPORTED = ("lh_config_check", "lh_subseq_len", "lh_total_entries", "lh_pooled_rows",
+            "lh_workspace_bytes", "lh_saved_offsets", "lh_pyramid", "lh_score_topk", "lh_gather",
+            "lh_attn_fwd", "lh_attn_bwd", "lh_scatter", "lh_scatter_bwd", "lh_gather_bwd",
+            "lh_forward", "lh_backward", "lh_get_device_status", "lh_status_string",
+            "lh_forward_launches", "lh_backward_launches")
+
+
+def make_config(B, N, H, d, L, p, k, scale: float = 0.0, scatter_mode: int = 0) -> lh_config:
+    return lh_config(B, N, H, d, L, p, k, scale, scatter_mode, 0)
+
+
+def _ck(code: int, where: str):
+    if code != LH_OK:
+        raise LighthouseError(code, where)
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _p(t: torch.Tensor | None, dtype=None, numel=None, name="tensor"):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if numel is not None and t.numel() * t.element_size() < numel:
+        raise ValueError(f"{name} holds {t.numel() * t.element_size()} bytes, needs {numel}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+BF16, F32, I32 = torch.bfloat16, torch.float32, torch.int32
+
+
+# ------------------------------------------------------------------ sizes --
+
+def lh_config_check(cfg: lh_config) -> int:
+    return _lib.lh_config_check(ctypes.byref(cfg))
+
+
+def lh_subseq_len(cfg: lh_config) -> int:
+    return _lib.lh_subseq_len(ctypes.byref(cfg))
+
+
+def lh_total_entries(cfg: lh_config) -> int:
+    return _lib.lh_total_entries(ctypes.byref(cfg))
+
+
+def lh_pooled_rows(cfg: lh_config) -> int:
+    return _lib.lh_pooled_rows(ctypes.byref(cfg))
+
+
+def lh_workspace_bytes(cfg: lh_config):
+    f, b, s = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _ck(_lib.lh_workspace_bytes(ctypes.byref(cfg), ctypes.byref(f), ctypes.byref(b),
+                                ctypes.byref(s)), "lh_workspace_bytes")
+    return f.value, b.value, s.value
+
+
+def lh_saved_offsets(cfg: lh_config):
+    arr = (ctypes.c_size_t * 7)()
+    _ck(_lib.lh_saved_offsets(ctypes.byref(cfg), arr), "lh_saved_offsets")
+    return list(arr)
+
+
+def lh_forward_launches(cfg: lh_config) -> int:
+    return _lib.lh_forward_launches(ctypes.byref(cfg))
+
+
+def lh_backward_launches(cfg: lh_config) -> int:
+    return _lib.lh_backward_launches(ctypes.byref(cfg))
+
+
+# ------------------------------------------------------------------ stages --
+
+def lh_pyramid(cfg, q, k, v, q_lv, k_lv, v_lv, qk, kq, stream=None):
+    _ck(_lib.lh_pyramid(ctypes.byref(cfg), _p(q, BF16, name="q"), _p(k, BF16, name="k"),
+                        _p(v, BF16, name="v"), _p(q_lv, BF16), _p(k_lv, BF16), _p(v_lv, BF16),
+                        _p(qk, F32), _p(kq, F32), _stream(stream)), "lh_pyramid")
+
+
+def lh_score_topk(cfg, qk, kq, sel_idx, slot_map, ws, stream=None):
+    _ck(_lib.lh_score_topk(ctypes.byref(cfg), _p(qk, F32), _p(kq, F32), _p(sel_idx, I32),
+                           _p(slot_map, I32), _p(ws), ws.numel() * ws.element_size(),
+                           _stream(stream)), "lh_score_topk")
+
+
+def lh_gather(cfg, q, k, v, q_lv, k_lv, v_lv, sel_idx, qg, kg, vg, stream=None):
+    _ck(_lib.lh_gather(ctypes.byref(cfg), _p(q, BF16), _p(k, BF16), _p(v, BF16), _p(q_lv, BF16),
+                       _p(k_lv, BF16), _p(v_lv, BF16), _p(sel_idx, I32), _p(qg, BF16),
+                       _p(kg, BF16), _p(vg, BF16), _stream(stream)), "lh_gather")
+
+
+def lh_attn_fwd(cfg, qg, kg, vg, og, lse, stream=None):
+    _ck(_lib.lh_attn_fwd(ctypes.byref(cfg), _p(qg, BF16), _p(kg, BF16), _p(vg, BF16),
+                         _p(og, BF16), _p(lse, F32), _stream(stream)), "lh_attn_fwd")
+
+
+def lh_attn_bwd(cfg, qg, kg, vg, og, lse, dog, dqg, dkg, dvg, ws, stream=None):
+    _ck(_lib.lh_attn_bwd(ctypes.byref(cfg), _p(qg, BF16), _p(kg, BF16), _p(vg, BF16),
+                         _p(og, BF16), _p(lse, F32), _p(dog, BF16), _p(dqg, BF16), _p(dkg, BF16),
+                         _p(dvg, BF16), _p(ws), ws.numel() * ws.element_size(),
+                         _stream(stream)), "lh_attn_bwd")
+
+
+def lh_scatter(cfg, og, slot_map, o, ws=None, stream=None):
+    nb = 0 if ws is None else ws.numel() * ws.element_size()
+    _ck(_lib.lh_scatter(ctypes.byref(cfg), _p(og, BF16), _p(slot_map, I32), _p(o, BF16),
+                        _p(ws), nb, _stream(stream)), "lh_scatter")
+
+
+def lh_scatter_bwd(cfg, dout, og, sel_idx, dog, delta, stream=None):
+    _ck(_lib.lh_scatter_bwd(ctypes.byref(cfg), _p(dout, BF16), _p(og, BF16), _p(sel_idx, I32),
+                            _p(dog, BF16), _p(delta, F32), _stream(stream)), "lh_scatter_bwd")
+
+
+def lh_gather_bwd(cfg, dqg, dkg, dvg, slot_map, dq, dk, dv, stream=None):
+    _ck(_lib.lh_gather_bwd(ctypes.byref(cfg), _p(dqg, BF16), _p(dkg, BF16), _p(dvg, BF16),
+                           _p(slot_map, I32), _p(dq, BF16), _p(dk, BF16), _p(dv, BF16),
+                           _stream(stream)), "lh_gather_bwd")
+
+
+def lh_forward(cfg, q, k, v, o, saved, ws, stream=None):
+    _ck(_lib.lh_forward(ctypes.byref(cfg), _p(q, BF16), _p(k, BF16), _p(v, BF16), _p(o, BF16),
+                        _p(saved), saved.numel() * saved.element_size(), _p(ws),
+                        ws.numel() * ws.element_size(), _stream(stream)), "lh_forward")
+
+
+def lh_backward(cfg, saved, dout, dq, dk, dv, ws, stream=None):
+    _ck(_lib.lh_backward(ctypes.byref(cfg), _p(saved), saved.numel() * saved.element_size(),
+                         _p(dout, BF16), _p(dq, BF16), _p(dk, BF16), _p(dv, BF16), _p(ws),
+                         ws.numel() * ws.element_size(), _stream(stream)), "lh_backward")
+
+
+def lh_get_device_status(stream=None):
+    detail = ctypes.c_int32(0)
+    code = _lib.lh_get_device_status(_stream(stream), ctypes.byref(detail))
+    return code, detail.value
+
+
+def check_device_status(stream=None):
+    code, detail = lh_get_device_status(stream)
+    if code != LH_OK:
+        raise LighthouseError(code, f"device status (detail {detail})")
+
+
+# ------------------------------------------------------- buffer helpers --
+
+def saved_views(cfg: lh_config, saved: torch.Tensor) -> dict:
+    """Typed views into the saved buffer of lh_forward (no copies)."""
+    off = lh_saved_offsets(cfg)
+    B, H, d = cfg.B, cfg.H, cfg.d
+    S, P = lh_subseq_len(cfg), lh_total_entries(cfg)
+
+    def view(i, dtype, shape):
+        n = 1
+        for s in shape:
+            n *= s
+        nbytes = n * torch.tensor([], dtype=dtype).element_size()
+        return saved[off[i]:off[i] + nbytes].view(dtype).view(*shape)
+
+    return dict(sel_idx=view(0, I32, (B, H, S)), slot_map=view(1, I32, (B, H, P)),
+                qg=view(2, BF16, (B, H, S, d)), kg=view(3, BF16, (B, H, S, d)),
+                vg=view(4, BF16, (B, H, S, d)), og=view(5, BF16, (B, H, S, d)),
+                lse=view(6, F32, (B, H, S)))
+
+
+class LighthouseLayer:
+    """Owns the saved and scratch buffers of one layer shape on one device.
+
+    forward(q, k, v) -> o and backward(dout) -> (dq, dk, dv) call lh_forward and
+    lh_backward on torch's current stream; tensors are [B, N, H, d] bf16.
+    """
+
+    def __init__(self, B, N, H, d, L, p, k, scale: float = 0.0, scatter_mode: int = 0,
+                 device="cuda"):
+        self.cfg = make_config(B, N, H, d, L, p, k, scale, scatter_mode)
+        _ck(lh_config_check(self.cfg), "lh_config_check")
+        fwd, bwd, saved = lh_workspace_bytes(self.cfg)
+        self.device = torch.device(device)
+        self.saved = torch.empty(saved, dtype=torch.uint8, device=self.device)
+        self.ws_fwd = torch.empty(fwd, dtype=torch.uint8, device=self.device)
+        self.ws_bwd = torch.empty(bwd, dtype=torch.uint8, device=self.device)
+        self.S = lh_subseq_len(self.cfg)
+
+    def forward(self, q, k, v, out=None):
+        o = torch.empty_like(q) if out is None else out
+        lh_forward(self.cfg, q, k, v, o, self.saved, self.ws_fwd)
+        return o
+
+    def backward(self, dout, grads=None):
+        if grads is None:
+            grads = tuple(torch.empty_like(dout) for _ in range(3))
+        lh_backward(self.cfg, self.saved, dout, *grads, self.ws_bwd)
+        return grads
+
+    def views(self):
+        return saved_views(self.cfg, self.saved)
+
+
+class LighthouseAttention(torch.autograd.Function):
+    """Autograd wrapper: y = Lighthouse(q, k, v); the selection is not differentiated."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, layer: LighthouseLayer):
+        ctx.layer = layer
+        return layer.forward(q.contiguous(), k.contiguous(), v.contiguous())
+
+    @staticmethod
+    def backward(ctx, dout):
+        dq, dk, dv = ctx.layer.backward(dout.contiguous())
+        return dq, dk, dv, None

@@ -1,0 +1,208 @@
+/*
+ * lighthouse.h - C ABI of the Lighthouse Attention layer's hot path on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method is the one of "Long Context Pre-Training with Lighthouse
+ * Attention" (arXiv 2605.06554): a four-stage pipeline that replaces causal
+ * scaled dot-product attention (Sec. 3.2):
+ *   (i)   symmetric mean pooling of per-head Q, K, V into an L-level pyramid
+ *         with pooling factor p (Sec. 3.3);
+ *   (ii)  parameter-free scores (per-head l2 norms at level 0, max-pooled at
+ *         coarser levels) and one joint top-k over the QK and KQ streams
+ *         (Sec. 3.4);
+ *   (iii) a gather of the selected (Q, K, V) triples into a contiguous
+ *         sub-sequence of length S = N/p^(L-1) + (L-1) p k, ordered so that a
+ *         plain S x S causal mask applies, and dense causal softmax attention
+ *         over it (Sec. 3.5, Eq. 8 and 9);
+ *   (iv)  a scatter of each output back to the base positions it represents,
+ *         shifted by p^l - 1 (Sec. 3.6);
+ * plus the backward of (iv), (iii) and the gather/pooling into dQ, dK, dV
+ * (Sec. 3.2: the selection itself carries no gradient).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - bf16 tensors are passed as lh_bf16 (the raw 16-bit pattern).  Token
+ *   tensors are [B, N, H, d] row-major; gathered tensors are [B, H, S, d];
+ *   per-entry arrays are [B, H, P] with P = sum_{l<L} N / p^l and the flat
+ *   pyramid index f(l, i) = sum_{l'<l} N/p^l' + i.
+ * - Every pointer that a kernel touches is a device pointer on the current
+ *   device, 16-byte aligned, and the buffers must not overlap.  The caller
+ *   owns all memory: no entry point allocates, frees or synchronises, except
+ *   lh_get_device_status, which synchronises the given stream.
+ * - `stream` is a cudaStream_t (passed as void*; NULL = legacy stream).  All
+ *   work is enqueued on it, asynchronously.
+ * - Errors: argument errors are reported synchronously, before any launch
+ *   (LH_ERR_INVALID_ARGUMENT, LH_ERR_UNSUPPORTED, LH_ERR_WORKSPACE).  A
+ *   failed launch returns LH_ERR_CUDA.  Errors found on the device (a wait
+ *   that ran out, an index out of range) are recorded in a device status word
+ *   that lh_get_device_status reads and clears.
+ * - Determinism: the same inputs give the same output bits, run after run.
+ * - Inputs must be finite.
+ */
+#ifndef LIGHTHOUSE_H
+#define LIGHTHOUSE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t lh_bf16; /* bit pattern of a bfloat16 value */
+
+typedef enum {
+  LH_OK = 0,
+  LH_ERR_INVALID_ARGUMENT = 1, /* bad pointer, size or config */
+  LH_ERR_UNSUPPORTED = 2,      /* valid for the method, not built here (e.g. d) */
+  LH_ERR_WORKSPACE = 3,        /* workspace or saved buffer too small */
+  LH_ERR_CUDA = 4,             /* a CUDA launch or driver call failed */
+  LH_ERR_DEVICE_TIMEOUT = 5,   /* a bounded device-side wait ran out */
+  LH_ERR_DEVICE_BOUNDS = 6     /* a device-side index check failed */
+} lh_status;
+
+/* One layer call.  Sec. 3.3 requires p^(L-1) | N; the budget (L-1) p k must
+ * not exceed the finer-level entry count.  scale <= 0 selects 1/sqrt(d).
+ * scatter_mode: 0 = gather-side (pull) scatter; 1 = fixed-point integer
+ * atomic scatter (same placement, order-independent sums).
+ * select_mode: 0 = one joint top-k over all finer levels (the only mode). */
+typedef struct {
+  int64_t B, N, H, d, L, p, k;
+  float scale;
+  int32_t scatter_mode;
+  int32_t select_mode;
+} lh_config;
+
+/* Returns LH_OK when the config is valid and supported: B, N, H >= 1,
+ * p >= 2, 1 <= L <= 8, p^(L-1) | N, 0 <= (L-1) p k <= sum_{l<L-1} N/p^l,
+ * d in {64, 128}, every index fits in int32 per (b, h). */
+lh_status lh_config_check(const lh_config* cfg);
+
+/* S = N/p^(L-1) + (L-1) p k (Sec. 3.5, Eq. 8); -1 for an invalid config. */
+int64_t lh_subseq_len(const lh_config* cfg);
+
+/* P = sum_{l=0}^{L-1} N / p^l, entries per (b, h) (Sec. 3.3); -1 if invalid. */
+int64_t lh_total_entries(const lh_config* cfg);
+
+/* Pooled rows per batch row: sum_{l=1}^{L-1} N / p^l; -1 if invalid. */
+int64_t lh_pooled_rows(const lh_config* cfg);
+
+/* Byte sizes of the caller-owned buffers:
+ *  fwd_ws  - scratch of lh_forward and lh_score_topk;
+ *  bwd_ws  - scratch of lh_backward and lh_attn_bwd;
+ *  saved   - what lh_forward leaves for lh_backward (see lh_saved_offsets).
+ * Any output pointer may be NULL. */
+lh_status lh_workspace_bytes(const lh_config* cfg, size_t* fwd_ws, size_t* bwd_ws,
+                             size_t* saved);
+
+/* Byte offsets inside the saved buffer, in this order: sel_idx (int32
+ * [B,H,S]), slot_map (int32 [B,H,P]), qg, kg, vg, og (bf16 [B,H,S,d]),
+ * lse (fp32 [B,H,S]).  `offsets` has room for 7 values. */
+lh_status lh_saved_offsets(const lh_config* cfg, size_t* offsets);
+
+/* (i) + the level-0/coarse scores of (ii), in one pass over Q, K, V.
+ * Sec. 3.3: level l, entry i = mean of base rows i p^l .. (i+1) p^l - 1.
+ * Sec. 3.4: qk/kq at level 0 are ||Q_t||_2 and ||K_t||_2 (squares summed in
+ * fp64, fp64 square root, rounded once to fp32); at level l they are the max
+ * of the level-0 scores in the window.
+ *  q, k, v        in  bf16 [B, N, H, d]
+ *  q_lv,k_lv,v_lv out bf16, levels 1..L-1 back to back; level l is
+ *                     [B, N/p^l, H, d] and starts after the rows of levels
+ *                     1..l-1 (lh_pooled_rows rows per batch row in total);
+ *                     may be NULL when L == 1
+ *  qk, kq         out fp32 [B, H, P]                                      */
+lh_status lh_pyramid(const lh_config* cfg, const lh_bf16* q, const lh_bf16* k,
+                     const lh_bf16* v, lh_bf16* q_lv, lh_bf16* k_lv, lh_bf16* v_lv,
+                     float* qk, float* kq, void* stream);
+
+/* (ii) joint top-k and the topological order of (iii), Sec. 3.4-3.5.
+ * Exactly (L-1) p k entries of levels 0..L-2 are chosen per (b, h) by the
+ * key r = max(qk, kq), descending, ties to the lower flat index; all of
+ * level L-1 is added.  Entries are ordered by their last base token
+ * e = (i+1) p^l - 1, then by level.
+ *  sel_idx  out int32 [B, H, S]  flat pyramid index of each slot
+ *  slot_map out int32 [B, H, P]  slot of each entry, -1 if not selected
+ *  ws       scratch of at least fwd_ws bytes (lh_workspace_bytes)          */
+lh_status lh_score_topk(const lh_config* cfg, const float* qk, const float* kq,
+                        int32_t* sel_idx, int32_t* slot_map, void* ws, size_t ws_bytes,
+                        void* stream);
+
+/* (iii) gather: row m of qg/kg/vg is the pyramid entry sel_idx[m]
+ * (level 0 from q/k/v, coarser levels from q_lv/k_lv/v_lv).
+ *  qg, kg, vg out bf16 [B, H, S, d]                                        */
+lh_status lh_gather(const lh_config* cfg, const lh_bf16* q, const lh_bf16* k,
+                    const lh_bf16* v, const lh_bf16* q_lv, const lh_bf16* k_lv,
+                    const lh_bf16* v_lv, const int32_t* sel_idx, lh_bf16* qg,
+                    lh_bf16* kg, lh_bf16* vg, void* stream);
+
+/* (iii) causal softmax attention over the gathered sub-sequence (Eq. 9):
+ * og[m] = sum_{m' <= m} softmax(scale qg[m].kg[m']) vg[m'], lse[m] = natural
+ * log of the softmax normaliser.  tcgen05 tensor cores, fp32 accumulation.
+ *  qg, kg, vg in  bf16 [B, H, S, d];  og out bf16 [B, H, S, d];
+ *  lse out fp32 [B, H, S]                                                  */
+lh_status lh_attn_fwd(const lh_config* cfg, const lh_bf16* qg, const lh_bf16* kg,
+                      const lh_bf16* vg, lh_bf16* og, float* lse, void* stream);
+
+/* Backward of lh_attn_fwd: with P the softmax rows, D = rowsum(dog * og),
+ * dS = P (dog vg^T - D): dqg = scale dS kg, dkg = scale dS^T qg,
+ * dvg = P^T dog.  Deterministic (no floating-point atomics).
+ *  ws scratch of at least bwd_ws bytes.                                    */
+lh_status lh_attn_bwd(const lh_config* cfg, const lh_bf16* qg, const lh_bf16* kg,
+                      const lh_bf16* vg, const lh_bf16* og, const float* lse,
+                      const lh_bf16* dog, lh_bf16* dqg, lh_bf16* dkg, lh_bf16* dvg,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/* (iv) scatter-back, Sec. 3.6: o[t] = sum over levels l of og[slot] for the
+ * selected entry (l, i) with (i+1) p^l - 1 <= t <= (i+2) p^l - 2, i.e.
+ * i = floor((t+1)/p^l) - 1; levels are summed in ascending order in fp32 and
+ * rounded once; a position no entry reaches gets 0.
+ *  o out bf16 [B, N, H, d].  scatter_mode 1 needs ws (fwd_ws bytes).      */
+lh_status lh_scatter(const lh_config* cfg, const lh_bf16* og, const int32_t* slot_map,
+                     lh_bf16* o, void* ws, size_t ws_bytes, void* stream);
+
+/* Adjoint of lh_scatter: dog[m] = sum of dO[t] over the shifted range of
+ * slot m (clipped to t < N), and delta[m] = rowsum(dog[m] * og[m]) (the D of
+ * the attention backward), both per (b, h).
+ *  dout in bf16 [B, N, H, d]; dog out bf16 [B, H, S, d]; delta out fp32
+ *  [B, H, S]                                                               */
+lh_status lh_scatter_bwd(const lh_config* cfg, const lh_bf16* dout, const lh_bf16* og,
+                         const int32_t* sel_idx, lh_bf16* dog, float* delta, void* stream);
+
+/* Adjoint of the gather and the mean pooling: dq[t] = sum over levels l of
+ * p^-l dqg[slot(l, floor(t/p^l))] for selected entries (unshifted window),
+ * likewise dk and dv.
+ *  dq, dk, dv out bf16 [B, N, H, d]                                        */
+lh_status lh_gather_bwd(const lh_config* cfg, const lh_bf16* dqg, const lh_bf16* dkg,
+                        const lh_bf16* dvg, const int32_t* slot_map, lh_bf16* dq,
+                        lh_bf16* dk, lh_bf16* dv, void* stream);
+
+/* Whole layer forward: lh_pyramid, lh_score_topk, lh_gather, lh_attn_fwd,
+ * lh_scatter.  o out bf16 [B, N, H, d].  `saved` (>= saved bytes) receives
+ * what lh_backward needs; `ws` (>= fwd_ws bytes) is scratch.               */
+lh_status lh_forward(const lh_config* cfg, const lh_bf16* q, const lh_bf16* k,
+                     const lh_bf16* v, lh_bf16* o, void* saved, size_t saved_bytes,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/* Whole layer backward from the saved buffer of the matching lh_forward:
+ * lh_scatter_bwd, lh_attn_bwd, lh_gather_bwd.  dq, dk, dv out bf16
+ * [B, N, H, d]; `ws` (>= bwd_ws bytes) is scratch.                          */
+lh_status lh_backward(const lh_config* cfg, const void* saved, size_t saved_bytes,
+                      const lh_bf16* dout, lh_bf16* dq, lh_bf16* dk, lh_bf16* dv,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, returns the first device-side error recorded since
+ * the last call (LH_OK if none) and clears it.  *detail (may be NULL)
+ * receives a kernel-specific code locating the failure. */
+lh_status lh_get_device_status(void* stream, int32_t* detail);
+
+/* Human-readable name of a status code (static string). */
+const char* lh_status_string(lh_status s);
+
+/* Number of kernel launches one lh_forward / lh_backward call makes. */
+int32_t lh_forward_launches(const lh_config* cfg);
+int32_t lh_backward_launches(const lh_config* cfg);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LIGHTHOUSE_H */

@@ -1,0 +1,45 @@
+"""Helpers shared by the GPU parity tests: tolerances and the per-head
+bridge between torch tensors and the oracle's numpy arrays."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+# Floating-point bar for bf16 outputs and gradients: max-abs 2e-2 and
+# rel-L2 5e-3.  The max-abs bound is applied to |x - y| / max(1, |y|): bf16
+# storage alone rounds by up to 2^-9 |y|, which passes 2e-2 in absolute
+# terms once |y| > 10, and outputs here reach |y| ~ 50 (heavy tokens).
+MAX_ABS = 2e-2
+REL_L2 = 5e-3
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def close_report(got, want):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    err = np.abs(got - want)
+    scaled = float(np.max(err / np.maximum(1.0, np.abs(want)))) if err.size else 0.0
+    rel = float(np.linalg.norm(err) / max(np.linalg.norm(want), 1e-30)) if err.size else 0.0
+    return scaled, rel
+
+
+def assert_close(got, want, name, max_abs=MAX_ABS, rel_l2=REL_L2):
+    scaled, rel = close_report(got, want)
+    assert np.all(np.isfinite(got)), f"{name}: non-finite values"
+    assert scaled <= max_abs and rel <= rel_l2, f"{name}: max-abs(scaled) {scaled:.3e}, rel-L2 {rel:.3e}"
+    return scaled, rel
+
+
+def bf16_ulp(x):
+    """One unit in the last place of bf16 at |x| (x != 0), as fp64."""
+    x = np.abs(np.asarray(x, dtype=np.float64))
+    _, e = np.frexp(np.where(x > 0, x, 1.0))
+    return np.ldexp(1.0, np.maximum(e - 8, -133))
+
+
+def head(x: torch.Tensor, b: int, h: int) -> np.ndarray:
+    """[B, N, H, d] tensor -> one head's [N, d] fp64 array."""
+    return np.ascontiguousarray(x[b, :, h, :].to(torch.float64).cpu().numpy())

@@ -1,0 +1,79 @@
+"""The C ABI library loads, exports every symbol the header declares, and its
+host-side size and config logic agrees with the oracle's formulas (no GPU
+needed: none of these calls launches a kernel)."""
+import os
+import re
+import subprocess
+
+import pytest
+
+from oracle import lighthouse_oracle as lo
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lighthouse.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from hierarchical_selection_attention_b200 import build
+    build.build()
+    from hierarchical_selection_attention_b200 import lighthouse
+    return lighthouse
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lh_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_and_library_exports_agree(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", L.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (lh_[a-z0-9_]+)", out))
+    decl = declared_symbols()
+    assert decl, "no declarations parsed"
+    missing = [s for s in decl if s not in exported]
+    assert not missing, missing
+    assert set(L.EXPORTED) == set(decl)
+
+
+@pytest.mark.parametrize("B,N,H,d,Lv,p,k", [(1, 4096, 2, 64, 3, 4, 64), (1, 65536, 8, 128, 3, 4, 1024),
+                                            (2, 131072, 8, 128, 3, 4, 2048),
+                                            (1, 524288, 8, 128, 3, 4, 4096),
+                                            (1, 1048576, 8, 128, 4, 4, 4096),
+                                            (3, 2048, 3, 128, 3, 4, 40), (1, 640, 2, 128, 1, 4, 0),
+                                            (1, 729, 1, 64, 4, 3, 5)])
+def test_sizes_match_oracle(L, B, N, H, d, Lv, p, k):
+    cfg = L.make_config(B, N, H, d, Lv, p, k)
+    assert L.lh_config_check(cfg) == 0
+    assert L.lh_subseq_len(cfg) == lo.subseq_len(N, Lv, p, k)
+    assert L.lh_total_entries(cfg) == lo.total_entries(N, Lv, p)
+    assert L.lh_pooled_rows(cfg) == lo.total_entries(N, Lv, p) - N
+    fwd, bwd, saved = L.lh_workspace_bytes(cfg)
+    S, P = lo.subseq_len(N, Lv, p, k), lo.total_entries(N, Lv, p)
+    assert saved >= B * H * (S * 4 + P * 4 + 4 * S * d * 2 + S * 4)
+    offs = L.lh_saved_offsets(cfg)
+    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+    assert bwd >= B * H * S * (4 * d * 2 + 4)
+    assert fwd >= 2 * B * H * P * 4 + 3 * B * (P - N) * H * d * 2
+
+
+@pytest.mark.parametrize("args,code", [
+    ((1, 100, 2, 64, 3, 4, 1), 1),      # 16 does not divide 100
+    ((1, 64, 2, 64, 3, 4, 100), 1),     # budget larger than the candidates
+    ((1, 64, 2, 96, 3, 4, 1), 2),       # head dim not built
+    ((1, 64, 2, 64, 3, 1, 1), 1),       # p < 2
+    ((0, 64, 2, 64, 3, 4, 1), 1),       # empty batch
+    ((1, 4096, 2, 64, 7, 2, 1), 2),     # more levels than built
+])
+def test_config_rejections(L, args, code):
+    assert L.lh_config_check(L.make_config(*args)) == code
+    assert L.lh_subseq_len(L.make_config(*args)) == -1
+
+
+def test_launch_counts(L):
+    cfg = L.make_config(1, 4096, 2, 64, 3, 4, 64)
+    assert L.lh_forward_launches(cfg) > 5
+    assert L.lh_backward_launches(cfg) >= 3
+    assert L.lh_forward_launches(L.make_config(1, 100, 2, 64, 3, 4, 1)) == -1
