@@ -1,0 +1,440 @@
+#!/usr/bin/env python
+"""Throughput of the Lighthouse Attention layer's hot path on B200.
+
+One step = one pass of the whole hot path over one batch: pyramid + scores,
+joint top-k and order, gather, causal attention, scatter-back (forward) and
+scatter adjoint, attention backward (dK/dV and dQ), gather/pooling adjoint
+(backward).  The workload is the pages' single-B200 shape: B=1, H=8, d=128,
+N=524288, L=3, p=4, k=4096 (S=65536), bf16, seeded synthetic inputs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line on rank 0.  Under torchrun (N > 1) every rank runs its
+own full workload (weak scaling, no collective on the data path); the
+reported time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from hierarchical_selection_attention_b200.inputs import WORKLOADS, make_dout, make_qkv  # noqa: E402
+
+METRIC = "Lighthouse layer fwd & fwd+bwd tokens/s at N=512K on 1 B200; per-stage % roofline"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = 3          # n512k_l3_p4_k4096
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        return dict(hbm=j["hbm_gbs"], tf_burst=j["bf16_tflops"],
+                    tf_sust=j.get("bf16_tflops_sustained", j["bf16_tflops"]), src="measured")
+    return dict(hbm=6650.0, tf_burst=1590.0, tf_sust=1400.0, src="fallback")
+
+
+def sizes(w):
+    B, N, H, d, L, p, k = (w[x] for x in ("B", "N", "H", "d", "L", "p", "k"))
+    S = N // p ** (L - 1) + (L - 1) * p * k
+    P = sum(N // p**l for l in range(L))
+    R = P - N
+    C = sum(N // p**l for l in range(L - 1))
+    return B, N, H, d, L, p, k, S, P, R, C
+
+
+def algorithmic(w):
+    """Per-launch algorithmic bytes (HBM stages) and FLOPs (attention) of each
+    stage: the bytes the method must move at least once, the FLOPs of the
+    causal GEMMs over the S x S triangle (diagonal included)."""
+    B, N, H, d, L, p, k, S, P, R, C = sizes(w)
+    tok = B * N * H * d * 2          # one [B, N, H, d] bf16 tensor
+    gat = B * H * S * d * 2          # one [B, H, S, d] bf16 tensor
+    tri = B * H * d * S * (S + 1)    # one causal GEMM: sum over rows of 2 d (row + 1)
+    return {
+        "pyramid": ("hbm", 3 * tok + 3 * B * R * H * d * 2 + 2 * B * H * P * 4),
+        "select": ("hbm", 2 * B * H * C * 4 + B * H * S * 4 + B * H * P * 4),
+        "gather": ("hbm", 6 * gat + B * H * S * 4),
+        "attn_fwd": ("tensor", 2 * tri),
+        "scatter": ("hbm", gat + tok + B * H * P * 4),
+        "scatter_bwd": ("hbm", tok + 3 * gat + B * H * S * 4),
+        "attn_bwd_dkdv": ("tensor", 4 * tri),
+        "attn_bwd_dq": ("tensor", 1 * tri),    # dS K; S and dP are recomputed (2 more GEMMs)
+        "gather_bwd": ("hbm", 3 * gat + 3 * tok + B * H * P * 4),
+    }
+
+
+EXECUTED_GEMMS = {"attn_fwd": 2, "attn_bwd_dkdv": 4, "attn_bwd_dq": 3}
+
+
+class Clocks:
+    """nvidia-smi sampling while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def start(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "100"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.flush()
+        rows = [r.split(",") for r in open(self.f.name).read().strip().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_init():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws):
+    if ws > 1:
+        torch.distributed.barrier()
+
+
+# ---------------------------------------------------------------- our arm --
+
+def run_ours(args, w, ws, rank, local):
+    from hierarchical_selection_attention_b200 import lighthouse as L
+
+    B, N, H, d, Lv, p, k, S, P, R, C = sizes(w)
+    dev = torch.device("cuda", local)
+    qh, kh, vh = make_qkv(B, N, H, d, seed=args.workload)
+    doh = make_dout(B, N, H, d, seed=args.workload)
+    q, kk, v, dout = (t.to(dev) for t in (qh, kh, vh, doh))
+    cfg = L.make_config(B, N, H, d, Lv, p, k)
+    layer = L.LighthouseLayer(B, N, H, d, Lv, p, k, device=dev)
+    sv = layer.views()
+    e = lambda *s, dt=torch.bfloat16: torch.empty(*s, dtype=dt, device=dev)
+    fws, _, _ = L.lh_workspace_bytes(cfg)
+    ws_f = torch.empty(fws, dtype=torch.uint8, device=dev)
+    q_lv, k_lv, v_lv = (e(max(B * R * H * d, 1)) for _ in range(3))
+    qk, kq = e(B, H, P, dt=torch.float32), e(B, H, P, dt=torch.float32)
+    o = torch.empty_like(q)
+    dog, delta = e(B, H, S, d), e(B, H, S, dt=torch.float32)
+    dqg, dkg, dvg = (e(B, H, S, d) for _ in range(3))
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    stages = [
+        ("pyramid", lambda: L.lh_pyramid(cfg, q, kk, v, q_lv, k_lv, v_lv, qk, kq)),
+        ("select", lambda: L.lh_score_topk(cfg, qk, kq, sv["sel_idx"], sv["slot_map"], ws_f)),
+        ("gather", lambda: L.lh_gather(cfg, q, kk, v, q_lv, k_lv, v_lv, sv["sel_idx"], sv["qg"],
+                                       sv["kg"], sv["vg"])),
+        ("attn_fwd", lambda: L.lh_attn_fwd(cfg, sv["qg"], sv["kg"], sv["vg"], sv["og"], sv["lse"],
+                                           og_lo=sv["og_lo"])),
+        ("scatter", lambda: L.lh_scatter(cfg, sv["og"], sv["slot_map"], o)),
+        ("scatter_bwd", lambda: L.lh_scatter_bwd(cfg, dout, sv["og"], sv["sel_idx"], dog, delta,
+                                                 og_lo=sv["og_lo"])),
+        ("attn_bwd_dkdv", lambda: L.lh_attn_bwd_dkdv(cfg, sv["qg"], sv["kg"], sv["vg"], dog,
+                                                     sv["lse"], delta, dkg, dvg)),
+        ("attn_bwd_dq", lambda: L.lh_attn_bwd_dq(cfg, sv["qg"], sv["kg"], sv["vg"], dog, sv["lse"],
+                                                 delta, dqg)),
+        ("gather_bwd", lambda: L.lh_gather_bwd(cfg, dqg, dkg, dvg, sv["slot_map"], dq, dk, dv)),
+    ]
+    n_fwd = 5
+    stream = torch.cuda.current_stream(dev)
+
+    def step(evs=None):
+        if evs is not None:
+            evs[0].record(stream)
+        for i, (_, fn) in enumerate(stages):
+            fn()
+            if evs is not None:
+                evs[i + 1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    L.check_device_status()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
+           for _ in range(args.steps)]
+    clk = Clocks(local)
+    clk.start()
+    barrier(ws)
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for s in range(args.steps):
+        step(evs[s])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(ws)
+    clocks = clk.stop()
+    L.check_device_status()
+    total_ms = max_over_ranks(t0.elapsed_time(t1), ws)
+    stage_ms = {name: statistics.mean(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(args.steps))
+                for i, (name, _) in enumerate(stages)}
+    fwd_ms = statistics.mean(evs[s][0].elapsed_time(evs[s][n_fwd]) for s in range(args.steps))
+    fwd_ms = max_over_ranks(fwd_ms, ws)
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        pin = lambda t: t.pin_memory()
+        hq, hk, hv, hdo = (pin(t) for t in (qh, kh, vh, doh))
+        ho, hdq, hdk, hdv = (torch.empty_like(hq).pin_memory() for _ in range(4))
+
+        def e2e_step():
+            for dst, src in ((q, hq), (kk, hk), (v, hv), (dout, hdo)):
+                dst.copy_(src, non_blocking=True)
+            layer.forward(q, kk, v, out=o)
+            layer.backward(dout, grads=(dq, dk, dv))
+            for dst, src in ((ho, o), (hdq, dq), (hdk, dk), (hdv, dv)):
+                dst.copy_(src, non_blocking=True)
+
+        for _ in range(max(1, min(args.warmup, 2))):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        n_e2e = max(3, min(args.steps, 10))
+        barrier(ws)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(ws)
+        L.check_device_status()
+        e2e_ms = max_over_ranks(a.elapsed_time(b), ws) / n_e2e
+        nbytes = B * N * H * d * 2
+        e2e = {"value": ws * B * N / (e2e_ms / 1e3), "unit": UNIT, "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": 4 * nbytes, "d2h_bytes_per_step": 4 * nbytes,
+               "api": "lh_forward + lh_backward, pinned host buffers"}
+
+    # ---- roofline, per stage and for the dominant kernel
+    pk = peaks()
+    alg = algorithmic(w)
+    per_stage = {}
+    for name, ms in stage_ms.items():
+        bound, amount = alg[name]
+        if bound == "hbm":
+            ach = amount / (ms / 1e3) / 1e9
+            per_stage[name] = {"ms": round(ms, 4), "bound": "hbm", "GB/s": round(ach, 1),
+                               "frac": round(ach / pk["hbm"], 4), "algorithmic_bytes": amount}
+        else:
+            ach = amount / (ms / 1e3) / 1e12
+            one_gemm = alg["attn_fwd"][1] / 2
+            tc = EXECUTED_GEMMS[name] * one_gemm / (ms / 1e3) / 1e12
+            per_stage[name] = {"ms": round(ms, 4), "bound": "tensor", "TFLOP/s": round(ach, 1),
+                               "frac": round(ach / pk["tf_sust"], 4), "algorithmic_flops": amount,
+                               "executed_TFLOP/s": round(tc, 1)}
+    dom = max(stage_ms, key=stage_ms.get)
+    bound, amount = alg[dom]
+    if bound == "hbm":
+        ach = amount / (stage_ms[dom] / 1e3) / 1e9
+        roof = {"bound": "hbm", "kernel": dom, "achieved": round(ach, 1), "peak": pk["hbm"],
+                "unit": "GB/s", "frac": round(ach / pk["hbm"], 4), "traffic": None}
+    else:
+        ach = amount / (stage_ms[dom] / 1e3) / 1e12
+        roof = {"bound": "tensor", "kernel": dom, "achieved": round(ach, 1), "peak": pk["tf_sust"],
+                "unit": "TFLOP/s", "frac": round(ach / pk["tf_sust"], 4), "traffic": None}
+    roof["peak_source"] = f"{pk['src']} (bf16 sustained for tensor, copy for HBM)"
+    traffic = load_traffic(dom)
+    if traffic is not None:
+        roof["traffic"] = traffic
+
+    launches = args.steps * (L.lh_forward_launches(cfg) + L.lh_backward_launches(cfg))
+    ms_step = total_ms / args.steps
+    line = {
+        "metric": METRIC, "value": ws * B * N / (ms_step / 1e3), "unit": UNIT, "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded: N(0,1) x per-token lognormal(0,0.5), 64 heavy tokens x4)",
+        "config": {"workload": f"{w['name']}: B={B} N={N} H={H} d={d} L={Lv} p={p} k={k} S={S}",
+                   "step": "lh_forward + lh_backward stages (fwd+bwd)",
+                   "l2": "inputs larger than L2 (3 GiB of Q,K,V per step); no flush",
+                   "parallelism": f"replicas x{ws} (independent layers, no collective)"},
+        "fwd_tokens_per_s": ws * B * N / (fwd_ms / 1e3), "fwd_ms": fwd_ms,
+        "stages": per_stage, "roofline": roof, "e2e": e2e, "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    return line
+
+
+def load_traffic(kernel):
+    """Per-launch DRAM bytes of the dominant kernel from the committed ncu
+    summary (profiles/traffic.json), if it was captured for this kernel."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    j = json.load(open(p))
+    ent = j.get(kernel)
+    return None if ent is None else ent.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------- oracle timing --
+
+def oracle_sample(w, rows_per_head: int, seed: int):
+    """Time the CPU oracle on a bounded sample of the workload: one (b, h)
+    head over all N tokens (scores, selection, order, pyramid, gather,
+    scatter and both adjoints) plus the attention forward and backward of
+    `rows_per_head` query rows spread evenly over S; the attention part is
+    scaled by S / rows_per_head, and the head by H and B.  Returns
+    (tokens/s, seconds measured, description)."""
+    from oracle import lighthouse_oracle as lo
+
+    B, N, H, d, Lv, p, k, S, P, R, C = sizes(w)
+    q, kk, v = make_qkv(1, N, 1, d, seed=seed)
+    dout = make_dout(1, N, 1, d, seed=seed)
+    qh, kh, vh, doh = (x[0, :, 0, :].double().numpy() for x in (q, kk, v, dout))
+    scale = 1.0 / math.sqrt(d)
+    t0 = time.perf_counter()
+    sel = lo.select_head(qh, kh, Lv, p, k)
+    pyr = [lo.pyramid(x, Lv, p) for x in (qh, kh, vh)]
+    qg, kg, vg = (lo.gather_rows(lv, sel["sel_idx"], N, Lv, p) for lv in pyr)
+    dog = lo.scatter_bwd(doh, sel["sel_idx"], N, Lv, p)
+    t_lin = time.perf_counter() - t0
+    rows = np.linspace(0, S - 1, rows_per_head).astype(np.int64)
+    t1 = time.perf_counter()
+    og_rows, _ = lo.attention(qg, kg, vg, scale, rows=rows)
+    dqg, dkg, dvg = lo.attention_bwd(qg, kg, vg, dog, scale, rows=rows)
+    t_att = time.perf_counter() - t1
+    t2 = time.perf_counter()
+    og = np.zeros_like(qg)
+    og[rows] = og_rows
+    lo.scatter(og, sel["slot_map"], N, Lv, p)
+    for g in (dqg, dkg, dvg):
+        lo.pyramid_bwd(g, sel["slot_map"], N, Lv, p)
+    t_lin += time.perf_counter() - t2
+    head_s = t_lin + t_att * S / rows_per_head
+    tok_s = B * N / (head_s * H * B)
+    measured = time.perf_counter() - t0
+    desc = (f"one (b,h) head of {w['name']}: all N={N} tokens through scores/top-k/order/pyramid/"
+            f"gather/scatter/adjoints, attention fwd+bwd on {rows_per_head} of S={S} query rows "
+            f"(scaled by S/{rows_per_head}), times B*H={B * H} heads; measured {measured:.1f} s")
+    return tok_s, measured, desc
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def run_reference(args, w):
+    vals = []
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        tok_s, _, desc = oracle_sample(w, rows_per_head=args.ref_rows, seed=args.workload)
+        if i >= args.warmup:
+            vals.append(tok_s)
+    v = statistics.median(vals)
+    cores = blas_threads()
+    return {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * sizes(w)[0] * sizes(w)[1] / v,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded, same recipe)", "impl": "reference",
+            "config": {"workload": w["name"], "arm": "CPU fp64 oracle (numpy), host cores"},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-rows", type=int, default=32)
+    ap.add_argument("--cpu-rows", type=int, default=96)
+    args = ap.parse_args()
+    w = WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return
+        args.steps = min(args.steps, 5)
+        args.warmup = min(args.warmup, 1)
+        print(json.dumps(run_reference(args, w)), flush=True)
+        return
+
+    ws, rank, local = dist_init()
+    try:
+        line = run_ours(args, w, ws, rank, local)
+        if rank == 0:
+            if not args.no_cpu_baseline and ws == 1:
+                tok_s, _, desc = oracle_sample(w, rows_per_head=args.cpu_rows, seed=args.workload)
+                line["cpu_baseline"] = {"value": tok_s, "unit": UNIT, "cores": blas_threads(),
+                                        "kind": "oracle", "sample": desc}
+            print(json.dumps(line), flush=True)
+    finally:
+        if ws > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -109,18 +109,20 @@ FwdWs fwd_layout(const LhDims& D, int scatter_mode) {
   return w;
 }
 
+constexpr int kSaved = 8;  // sel_idx, slot_map, qg, kg, vg, og, og_lo, lse
+
 struct Saved {
-  size_t off[7];
+  size_t off[kSaved];
   size_t total;
 };
 
 Saved saved_layout(const LhDims& D) {
   Saved s;
   const size_t rows = (size_t)D.B * D.H * D.S;
-  const size_t sizes[7] = {rows * 4, (size_t)D.B * D.H * D.P * 4, rows * D.d * 2, rows * D.d * 2,
-                           rows * D.d * 2, rows * D.d * 2, rows * 4};
+  const size_t g = rows * D.d * 2;
+  const size_t sizes[kSaved] = {rows * 4, (size_t)D.B * D.H * D.P * 4, g, g, g, g, g, rows * 4};
   size_t o = 0;
-  for (int i = 0; i < 7; ++i) {
+  for (int i = 0; i < kSaved; ++i) {
     s.off[i] = o;
     o += up(sizes[i]);
   }
@@ -206,7 +208,7 @@ lh_status lh_saved_offsets(const lh_config* cfg, size_t* offsets) {
   LH_TRY(check(cfg));
   if (!offsets) return LH_ERR_INVALID_ARGUMENT;
   const Saved s = saved_layout(dims(cfg));
-  for (int i = 0; i < 7; ++i) offsets[i] = s.off[i];
+  for (int i = 0; i < kSaved; ++i) offsets[i] = s.off[i];
   return LH_OK;
 }
 
@@ -246,30 +248,55 @@ lh_status lh_gather(const lh_config* cfg, const lh_bf16* q, const lh_bf16* k,
 }
 
 lh_status lh_attn_fwd(const lh_config* cfg, const lh_bf16* qg, const lh_bf16* kg,
-                      const lh_bf16* vg, lh_bf16* og, float* lse, void* stream) {
+                      const lh_bf16* vg, lh_bf16* og, lh_bf16* og_lo, float* lse,
+                      void* stream) {
   LH_TRY(check(cfg));
   if (!all_aligned(qg, kg, vg, og, lse)) return LH_ERR_INVALID_ARGUMENT;
+  if (og_lo && !aligned(og_lo)) return LH_ERR_INVALID_ARGUMENT;
   const LhDims D = launch_dims(cfg);
   if (!D.status) return LH_ERR_CUDA;
-  return cu(lh_launch_attn_fwd(D.B * D.H, D.S, D.d, D.scale, qg, kg, vg, og, lse, D.status,
-                               (cudaStream_t)stream));
+  return cu(lh_launch_attn_fwd(D.B * D.H, D.S, D.d, D.scale, qg, kg, vg, og, og_lo, lse,
+                               D.status, (cudaStream_t)stream));
 }
 
 lh_status lh_attn_bwd(const lh_config* cfg, const lh_bf16* qg, const lh_bf16* kg,
-                      const lh_bf16* vg, const lh_bf16* og, const float* lse,
-                      const lh_bf16* dog, lh_bf16* dqg, lh_bf16* dkg, lh_bf16* dvg, void* ws,
-                      size_t ws_bytes, void* stream) {
+                      const lh_bf16* vg, const lh_bf16* og, const lh_bf16* og_lo,
+                      const float* lse, const lh_bf16* dog, lh_bf16* dqg, lh_bf16* dkg,
+                      lh_bf16* dvg, void* ws, size_t ws_bytes, void* stream) {
   LH_TRY(check(cfg));
   if (!all_aligned(qg, kg, vg, og, lse, dog, dqg, dkg, dvg, ws)) return LH_ERR_INVALID_ARGUMENT;
+  if (og_lo && !aligned(og_lo)) return LH_ERR_INVALID_ARGUMENT;
   const LhDims D = launch_dims(cfg);
   if (!D.status) return LH_ERR_CUDA;
   const BwdWs b = bwd_layout(D);
   if (ws_bytes < b.total) return LH_ERR_WORKSPACE;
   const cudaStream_t st = (cudaStream_t)stream;
   float* delta = at<float>(ws, b.delta);
-  LH_TRY(cu(lh_launch_attn_delta(D.B * D.H, D.S, D.d, og, dog, delta, st)));
+  LH_TRY(cu(lh_launch_attn_delta(D.B * D.H, D.S, D.d, og, og_lo, dog, delta, st)));
   return cu(lh_launch_attn_bwd(D.B * D.H, D.S, D.d, D.scale, qg, kg, vg, dog, lse, delta, dqg,
-                               dkg, dvg, D.status, st, nullptr));
+                               dkg, dvg, D.status, st, 3));
+}
+
+lh_status lh_attn_bwd_dkdv(const lh_config* cfg, const lh_bf16* qg, const lh_bf16* kg,
+                           const lh_bf16* vg, const lh_bf16* dog, const float* lse,
+                           const float* delta, lh_bf16* dkg, lh_bf16* dvg, void* stream) {
+  LH_TRY(check(cfg));
+  if (!all_aligned(qg, kg, vg, dog, lse, delta, dkg, dvg)) return LH_ERR_INVALID_ARGUMENT;
+  const LhDims D = launch_dims(cfg);
+  if (!D.status) return LH_ERR_CUDA;
+  return cu(lh_launch_attn_bwd(D.B * D.H, D.S, D.d, D.scale, qg, kg, vg, dog, lse, delta, nullptr,
+                               dkg, dvg, D.status, (cudaStream_t)stream, 1));
+}
+
+lh_status lh_attn_bwd_dq(const lh_config* cfg, const lh_bf16* qg, const lh_bf16* kg,
+                         const lh_bf16* vg, const lh_bf16* dog, const float* lse,
+                         const float* delta, lh_bf16* dqg, void* stream) {
+  LH_TRY(check(cfg));
+  if (!all_aligned(qg, kg, vg, dog, lse, delta, dqg)) return LH_ERR_INVALID_ARGUMENT;
+  const LhDims D = launch_dims(cfg);
+  if (!D.status) return LH_ERR_CUDA;
+  return cu(lh_launch_attn_bwd(D.B * D.H, D.S, D.d, D.scale, qg, kg, vg, dog, lse, delta, dqg,
+                               nullptr, nullptr, D.status, (cudaStream_t)stream, 2));
 }
 
 lh_status lh_scatter(const lh_config* cfg, const lh_bf16* og, const int32_t* slot_map,
@@ -287,12 +314,14 @@ lh_status lh_scatter(const lh_config* cfg, const lh_bf16* og, const int32_t* slo
 }
 
 lh_status lh_scatter_bwd(const lh_config* cfg, const lh_bf16* dout, const lh_bf16* og,
-                         const int32_t* sel_idx, lh_bf16* dog, float* delta, void* stream) {
+                         const lh_bf16* og_lo, const int32_t* sel_idx, lh_bf16* dog,
+                         float* delta, void* stream) {
   LH_TRY(check(cfg));
   if (!all_aligned(dout, og, sel_idx, dog, delta)) return LH_ERR_INVALID_ARGUMENT;
+  if (og_lo && !aligned(og_lo)) return LH_ERR_INVALID_ARGUMENT;
   const LhDims D = launch_dims(cfg);
   if (!D.status) return LH_ERR_CUDA;
-  return cu(lh_launch_scatter_bwd(D, dout, og, sel_idx, dog, delta, (cudaStream_t)stream));
+  return cu(lh_launch_scatter_bwd(D, dout, og, og_lo, sel_idx, dog, delta, (cudaStream_t)stream));
 }
 
 lh_status lh_gather_bwd(const lh_config* cfg, const lh_bf16* dqg, const lh_bf16* dkg,
@@ -322,7 +351,8 @@ lh_status lh_forward(const lh_config* cfg, const lh_bf16* q, const lh_bf16* k,
   lh_bf16* kg = at<lh_bf16>(saved, s.off[3]);
   lh_bf16* vg = at<lh_bf16>(saved, s.off[4]);
   lh_bf16* og = at<lh_bf16>(saved, s.off[5]);
-  float* lse = at<float>(saved, s.off[6]);
+  lh_bf16* og_lo = at<lh_bf16>(saved, s.off[6]);
+  float* lse = at<float>(saved, s.off[7]);
   lh_bf16* q_lv = at<lh_bf16>(ws, w.q_lv);
   lh_bf16* k_lv = at<lh_bf16>(ws, w.k_lv);
   lh_bf16* v_lv = at<lh_bf16>(ws, w.v_lv);
@@ -331,7 +361,8 @@ lh_status lh_forward(const lh_config* cfg, const lh_bf16* q, const lh_bf16* k,
   LH_TRY(cu(lh_launch_pyramid(D, q, k, v, q_lv, k_lv, v_lv, qk, kq, st)));
   LH_TRY(cu(lh_launch_select(D, qk, kq, sel_idx, slot_map, at<void>(ws, w.select), st, nullptr)));
   LH_TRY(cu(lh_launch_gather(D, q, k, v, q_lv, k_lv, v_lv, sel_idx, qg, kg, vg, st)));
-  LH_TRY(cu(lh_launch_attn_fwd(D.B * D.H, D.S, D.d, D.scale, qg, kg, vg, og, lse, D.status, st)));
+  LH_TRY(cu(lh_launch_attn_fwd(D.B * D.H, D.S, D.d, D.scale, qg, kg, vg, og, og_lo, lse, D.status,
+                               st)));
   if (cfg->scatter_mode == 1)
     return cu(lh_launch_scatter_atomic(D, og, slot_map, o, at<void>(ws, w.atomic), st, nullptr));
   return cu(lh_launch_scatter(D, og, slot_map, o, st));
@@ -354,15 +385,16 @@ lh_status lh_backward(const lh_config* cfg, const void* saved, size_t saved_byte
   const lh_bf16* kg = at<lh_bf16>(saved, s.off[3]);
   const lh_bf16* vg = at<lh_bf16>(saved, s.off[4]);
   const lh_bf16* og = at<lh_bf16>(saved, s.off[5]);
-  const float* lse = at<float>(saved, s.off[6]);
+  const lh_bf16* og_lo = at<lh_bf16>(saved, s.off[6]);
+  const float* lse = at<float>(saved, s.off[7]);
   lh_bf16* dog = at<lh_bf16>(ws, b.dog);
   float* delta = at<float>(ws, b.delta);
   lh_bf16* dqg = at<lh_bf16>(ws, b.dqg);
   lh_bf16* dkg = at<lh_bf16>(ws, b.dkg);
   lh_bf16* dvg = at<lh_bf16>(ws, b.dvg);
-  LH_TRY(cu(lh_launch_scatter_bwd(D, dout, og, sel_idx, dog, delta, st)));
+  LH_TRY(cu(lh_launch_scatter_bwd(D, dout, og, og_lo, sel_idx, dog, delta, st)));
   LH_TRY(cu(lh_launch_attn_bwd(D.B * D.H, D.S, D.d, D.scale, qg, kg, vg, dog, lse, delta, dqg,
-                               dkg, dvg, D.status, st, nullptr)));
+                               dkg, dvg, D.status, st, 3)));
   return cu(lh_launch_gather_bwd(D, dqg, dkg, dvg, slot_map, dq, dk, dv, st));
 }
 
@@ -394,8 +426,9 @@ const char* lh_status_string(lh_status s) {
 int32_t lh_forward_launches(const lh_config* cfg) {
   if (check(cfg) != LH_OK) return -1;
   const LhDims D = dims(cfg);
-  const int select = D.n_cand > 0 ? 12 + 1 + 3 : 1 + 1 + 3;  // memset + hist/find pairs + order
-  const int scatter = cfg->scatter_mode == 1 ? 3 : 1;
+  // kernels only (the memsets of the scratch are copy-engine work, not counted)
+  const int select = D.n_cand > 0 ? 12 + 3 : 1 + 3;  // hist/find pairs + order count/scan/emit
+  const int scatter = cfg->scatter_mode == 1 ? 2 : 1;
   return 1 + select + 1 + 1 + scatter;
 }
 

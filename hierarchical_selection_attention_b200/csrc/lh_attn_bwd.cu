@@ -1,11 +1,516 @@
-// Backward of the gathered causal attention (placeholder until the tcgen05
-// kernels land).
+// Backward of the gathered causal attention of Lighthouse Attention ("Long
+// Context Pre-Training with Lighthouse Attention", Sec. 3.2: gradients reach
+// Q, K, V through the scatter, the attention of Eq. 9 and the gather).
+//
+// With s = scale q.k, P = softmax rows (rebuilt from the saved LSE),
+// dP = dO V^T and D = rowsum(dO * O):  dS = P (dP - D), dV = P^T dO,
+// dK = scale dS^T Q, dQ = scale dS K.  Two tcgen05 kernels, neither with
+// floating-point atomics, so every gradient is bitwise reproducible:
+//
+//  k_attn_bwd_dkdv  one CTA per 128 key rows of one (b, h); walks the query
+//                   tiles of 64 rows at and after its diagonal.  TMEM holds
+//                   S^T and dP^T (two buffers each, 64 columns) and the dV,
+//                   dK accumulators (d columns each).
+//  k_attn_bwd_dq    one CTA per 128 query rows; walks the key tiles of 64
+//                   rows up to its diagonal, recomputing S and dP, and
+//                   accumulates dQ in TMEM.
+//
+// Warp roles as in the forward: warp 0 issues TMA loads (2-stage ring of the
+// walked tiles), warp 1 issues the MMAs from one thread and commits them to
+// mbarriers, warps 2-5 own one TMEM lane (= one row of the stationary tile)
+// each, turn scores into P and dS in fp32, and write them to shared memory
+// as bf16 in the 128-byte-swizzled K-major layout the gradient MMAs read.
+// The same shared-memory tile of Q, dO or K serves as a K-major operand in
+// one MMA and as an MN-major operand in another.
 #include "lh_sm100.cuh"
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ------------------------------------------------------------------ dK/dV --
+
+constexpr int KV_M = 128;  // stationary key rows
+constexpr int Q_N = 64;    // walked query rows per tile
+
+template <int HD>
+struct DkdvLayout {
+  static constexpr uint32_t k = 0;
+  static constexpr uint32_t v = k + KV_M * HD * 2;
+  static constexpr uint32_t q = v + KV_M * HD * 2;            // 2 stages
+  static constexpr uint32_t dO = q + 2 * Q_N * HD * 2;        // 2 stages
+  static constexpr uint32_t p = dO + 2 * Q_N * HD * 2;        // [128][64] bf16
+  static constexpr uint32_t ds = p + KV_M * Q_N * 2;          // [128][64] bf16
+  static constexpr uint32_t vec = ds + KV_M * Q_N * 2;        // lse/delta, 2 x 2 x 64 fp32
+  static constexpr uint32_t bar = vec + 4 * Q_N * 4;
+  static constexpr uint32_t bytes = bar + 256;
+};
+
+struct DkdvBars {
+  uint64_t kvfull, qfull[2], qempty[2], sfull[2], sfree[2], pfull, dsfree, done, lfull[2];
+  uint32_t tmem_base;
+};
+
+// Columns: S^T buffers 0/64, dP^T buffers 128/192, dV 256, dK 256 + HD.
+template <int HD>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_attn_bwd_dkdv(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                    const float* __restrict__ lse, const float* __restrict__ delta,
+                    uint4* __restrict__ dkg, uint4* __restrict__ dvg, int S, int BH, float scale,
+                    int* status) {
+  using Lay = DkdvLayout<HD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~(uintptr_t)1023);
+  DkdvBars* bars = reinterpret_cast<DkdvBars*>(smem + Lay::bar);
+  float* vec = reinterpret_cast<float*>(smem + Lay::vec);  // [buf][lse|delta][64]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kt = (int)(blockIdx.x / BH);  // key tile 0 walks the most query tiles: first
+  const int bh = (int)(blockIdx.x % BH);
+  const int n_q = (S + Q_N - 1) / Q_N;
+  const int i0 = kt * (KV_M / Q_N);  // first query tile at or after the diagonal
+  const int n_it = n_q - i0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->kvfull, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->qfull[s], 1);
+      mbar_init(&bars->qempty[s], 1);
+      mbar_init(&bars->sfull[s], 1);
+      mbar_init(&bars->sfree[s], 128);
+      mbar_init(&bars->lfull[s], Q_N);
+    }
+    mbar_init(&bars->pfull, 128);
+    mbar_init(&bars->dsfree, 1);
+    mbar_init(&bars->done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_expect_tx(&bars->kvfull, 2 * KV_M * HD * 2);
+      for (int blk = 0; blk < HD / 64; ++blk) {
+        tma_load_3d(&tmK, &bars->kvfull, smem + Lay::k + blk * KV_M * 128, 64 * blk, kt * KV_M, bh);
+        tma_load_3d(&tmV, &bars->kvfull, smem + Lay::v + blk * KV_M * 128, 64 * blk, kt * KV_M, bh);
+      }
+      for (int it = 0; it < n_it; ++it) {
+        const int s = it & 1;
+        if (!mbar_wait(&bars->qempty[s], ((it >> 1) & 1) ^ 1, status, 21)) break;
+        mbar_expect_tx(&bars->qfull[s], 2 * Q_N * HD * 2);
+        const int row = (i0 + it) * Q_N;
+        for (int blk = 0; blk < HD / 64; ++blk) {
+          tma_load_3d(&tmQ, &bars->qfull[s], smem + Lay::q + s * Q_N * HD * 2 + blk * Q_N * 128,
+                      64 * blk, row, bh);
+          tma_load_3d(&tmO, &bars->qfull[s], smem + Lay::dO + s * Q_N * HD * 2 + blk * Q_N * 128,
+                      64 * blk, row, bh);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(KV_M, Q_N, 0, 0);   // S^T, dP^T
+      constexpr uint32_t idG = idesc_bf16(KV_M, HD, 0, 1);    // dV, dK (B MN-major)
+      const uint32_t sK = smem_u32(smem + Lay::k), sV = smem_u32(smem + Lay::v);
+      const uint32_t sQ = smem_u32(smem + Lay::q), sO = smem_u32(smem + Lay::dO);
+      const uint32_t sP = smem_u32(smem + Lay::p), sDS = smem_u32(smem + Lay::ds);
+      bool ok = mbar_wait(&bars->kvfull, 0, status, 22);
+      auto grads = [&](int it) -> bool {
+        const int s = it & 1;
+        if (!mbar_wait(&bars->pfull, it & 1, status, 23)) return false;
+        tc_fence_after();
+        const uint32_t qb = sQ + s * Q_N * HD * 2, ob = sO + s * Q_N * HD * 2;
+#pragma unroll
+        for (int ks = 0; ks < Q_N / 16; ++ks) {
+          const uint64_t ap = sdesc_sw128(sP + ks * 32, 16, 1024);
+          const uint64_t ad = sdesc_sw128(sDS + ks * 32, 16, 1024);
+          const uint64_t bo = sdesc_sw128(ob + ks * 16 * 128, Q_N * 128, 1024);
+          const uint64_t bq = sdesc_sw128(qb + ks * 16 * 128, Q_N * 128, 1024);
+          const uint32_t acc = (it > 0 || ks > 0) ? 1u : 0u;
+          mma_bf16(tmem + 256, ap, bo, idG, acc);       // dV += P^T dO
+          mma_bf16(tmem + 256 + HD, ad, bq, idG, acc);  // dK += dS^T Q
+        }
+        mma_commit(&bars->dsfree);
+        mma_commit(&bars->qempty[s]);
+        return true;
+      };
+      for (int it = 0; ok && it < n_it; ++it) {
+        const int s = it & 1, sb = it & 1;
+        if (!mbar_wait(&bars->qfull[s], (it >> 1) & 1, status, 24)) { ok = false; break; }
+        if (!mbar_wait(&bars->sfree[sb], ((it >> 1) & 1) ^ 1, status, 25)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t qb = sQ + s * Q_N * HD * 2, ob = sO + s * Q_N * HD * 2;
+#pragma unroll
+        for (int ks = 0; ks < HD / 16; ++ks) {
+          const uint32_t koff = (ks >> 2) * KV_M * 128 + (ks & 3) * 32;
+          const uint32_t qoff = (ks >> 2) * Q_N * 128 + (ks & 3) * 32;
+          mma_bf16(tmem + sb * Q_N, sdesc_sw128(sK + koff, 16, 1024),
+                   sdesc_sw128(qb + qoff, 16, 1024), idS, ks > 0 ? 1u : 0u);
+          mma_bf16(tmem + 128 + sb * Q_N, sdesc_sw128(sV + koff, 16, 1024),
+                   sdesc_sw128(ob + qoff, 16, 1024), idS, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars->sfull[sb]);
+        if (it > 0 && !grads(it - 1)) { ok = false; break; }
+      }
+      if (ok && grads(n_it - 1)) mma_commit(&bars->done);
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;               // key row in the tile
+    const int kvrow = kt * KV_M + r;
+    const int st = threadIdx.x - 64;                 // 0..127 among the softmax threads
+    const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+    uint8_t* pP = smem + Lay::p;
+    uint8_t* pDS = smem + Lay::ds;
+    const float c = scale * kLog2e;
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      const int sb = it & 1;
+      const int q0 = (i0 + it) * Q_N;
+      // LSE (log2 units) and D of the tile's 64 query rows, shared through
+      // shared memory.  The buffer used two tiles ago is free: every reader
+      // arrived on pfull for that tile before this thread saw dsfree for it.
+      float* lbuf = vec + sb * 2 * Q_N;
+      if (st < Q_N) {
+        const int qr = q0 + st;
+        lbuf[st] = qr < S ? __ldg(lse + (int64_t)bh * S + qr) * kLog2e : INFINITY;
+        lbuf[Q_N + st] = qr < S ? __ldg(delta + (int64_t)bh * S + qr) : 0.f;
+        mbar_arrive(&bars->lfull[sb]);
+      }
+      if (!mbar_wait(&bars->lfull[sb], (it >> 1) & 1, status, 29)) { ok = false; break; }
+      if (!mbar_wait(&bars->sfull[sb], (it >> 1) & 1, status, 26)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sr[2][32], pr[2][32];
+      tmem_ld32(tmem + lane_addr + sb * Q_N, sr[0]);
+      tmem_ld32(tmem + lane_addr + sb * Q_N + 32, sr[1]);
+      tmem_ld32(tmem + lane_addr + 128 + sb * Q_N, pr[0]);
+      tmem_ld32(tmem + lane_addr + 128 + sb * Q_N + 32, pr[1]);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&bars->sfree[sb]);
+      const bool diag = q0 < kt * KV_M + KV_M;       // the tile crosses the diagonal
+      uint32_t pk[Q_N / 2], dk[Q_N / 2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int col = h * 32 + e;
+          float p0 = ex2(fmaf(__uint_as_float(sr[h][e]), c, -lbuf[col]));
+          float p1 = ex2(fmaf(__uint_as_float(sr[h][e + 1]), c, -lbuf[col + 1]));
+          if (diag) {
+            p0 = (q0 + col >= kvrow) ? p0 : 0.f;
+            p1 = (q0 + col + 1 >= kvrow) ? p1 : 0.f;
+          }
+          const float d0 = p0 * (__uint_as_float(pr[h][e]) - lbuf[Q_N + col]);
+          const float d1 = p1 * (__uint_as_float(pr[h][e + 1]) - lbuf[Q_N + col + 1]);
+          pk[col >> 1] = pack_bf16x2(p0, p1);
+          dk[col >> 1] = pack_bf16x2(d0, d1);
+        }
+      if (it > 0 && !mbar_wait(&bars->dsfree, (it - 1) & 1, status, 27)) { ok = false; break; }
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc) {
+        const uint32_t off = r * 128 + ((cc ^ (r & 7)) << 4);
+        *reinterpret_cast<uint4*>(pP + off) = make_uint4(pk[cc * 4], pk[cc * 4 + 1], pk[cc * 4 + 2], pk[cc * 4 + 3]);
+        *reinterpret_cast<uint4*>(pDS + off) = make_uint4(dk[cc * 4], dk[cc * 4 + 1], dk[cc * 4 + 2], dk[cc * 4 + 3]);
+      }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars->pfull);
+    }
+    if (ok && mbar_wait(&bars->done, 0, status, 28)) {
+      tc_fence_after();
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {     // 0: dV, 1: dK
+        uint4* dst = (which ? dkg : dvg) + ((int64_t)bh * S + kvrow) * (HD / 8);
+        const float mul = which ? scale : 1.f;
+#pragma unroll
+        for (int cchunk = 0; cchunk < HD / 32; ++cchunk) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_addr + 256 + which * HD + cchunk * 32, o);
+          tmem_ld_wait();
+          if (kvrow < S) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(o[v * 8 + 0]) * mul, __uint_as_float(o[v * 8 + 1]) * mul);
+              w.y = pack_bf16x2(__uint_as_float(o[v * 8 + 2]) * mul, __uint_as_float(o[v * 8 + 3]) * mul);
+              w.z = pack_bf16x2(__uint_as_float(o[v * 8 + 4]) * mul, __uint_as_float(o[v * 8 + 5]) * mul);
+              w.w = pack_bf16x2(__uint_as_float(o[v * 8 + 6]) * mul, __uint_as_float(o[v * 8 + 7]) * mul);
+              dst[cchunk * 4 + v] = w;
+            }
+          }
+        }
+      }
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// --------------------------------------------------------------------- dQ --
+
+constexpr int Q_M = 128;   // stationary query rows
+constexpr int KV_N = 64;   // walked key rows per tile
+
+template <int HD>
+struct DqLayout {
+  static constexpr uint32_t q = 0;
+  static constexpr uint32_t dO = q + Q_M * HD * 2;
+  static constexpr uint32_t k = dO + Q_M * HD * 2;          // 2 stages
+  static constexpr uint32_t v = k + 2 * KV_N * HD * 2;       // 2 stages
+  static constexpr uint32_t ds = v + 2 * KV_N * HD * 2;      // [128][64] bf16
+  static constexpr uint32_t bar = ds + Q_M * KV_N * 2;
+  static constexpr uint32_t bytes = bar + 256;
+};
+
+struct DqBars {
+  uint64_t qfull, kvfull[2], kvempty[2], sfull[2], sfree[2], pfull, dsfree, done;
+  uint32_t tmem_base;
+};
+
+// Columns: S buffers 0/64, dP buffers 128/192, dQ 256.
+template <int HD>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_attn_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                  const float* __restrict__ lse, const float* __restrict__ delta,
+                  uint4* __restrict__ dqg, int S, int BH, float scale, int* status) {
+  using Lay = DqLayout<HD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~(uintptr_t)1023);
+  DqBars* bars = reinterpret_cast<DqBars*>(smem + Lay::bar);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_qt = (S + Q_M - 1) / Q_M;
+  const int qt = n_qt - 1 - (int)(blockIdx.x / BH);  // longest rows first
+  const int bh = (int)(blockIdx.x % BH);
+  const int n_kv = min((qt * Q_M + Q_M) / KV_N, (S + KV_N - 1) / KV_N);
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->qfull, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->kvfull[s], 1);
+      mbar_init(&bars->kvempty[s], 1);
+      mbar_init(&bars->sfull[s], 1);
+      mbar_init(&bars->sfree[s], 128);
+    }
+    mbar_init(&bars->pfull, 128);
+    mbar_init(&bars->dsfree, 1);
+    mbar_init(&bars->done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_expect_tx(&bars->qfull, 2 * Q_M * HD * 2);
+      for (int blk = 0; blk < HD / 64; ++blk) {
+        tma_load_3d(&tmQ, &bars->qfull, smem + Lay::q + blk * Q_M * 128, 64 * blk, qt * Q_M, bh);
+        tma_load_3d(&tmO, &bars->qfull, smem + Lay::dO + blk * Q_M * 128, 64 * blk, qt * Q_M, bh);
+      }
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j & 1;
+        if (!mbar_wait(&bars->kvempty[s], ((j >> 1) & 1) ^ 1, status, 31)) break;
+        mbar_expect_tx(&bars->kvfull[s], 2 * KV_N * HD * 2);
+        for (int blk = 0; blk < HD / 64; ++blk) {
+          tma_load_3d(&tmK, &bars->kvfull[s], smem + Lay::k + s * KV_N * HD * 2 + blk * KV_N * 128,
+                      64 * blk, j * KV_N, bh);
+          tma_load_3d(&tmV, &bars->kvfull[s], smem + Lay::v + s * KV_N * HD * 2 + blk * KV_N * 128,
+                      64 * blk, j * KV_N, bh);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(Q_M, KV_N, 0, 0);   // S, dP
+      constexpr uint32_t idG = idesc_bf16(Q_M, HD, 0, 1);     // dQ (B = K, MN-major)
+      const uint32_t sQ = smem_u32(smem + Lay::q), sO = smem_u32(smem + Lay::dO);
+      const uint32_t sK = smem_u32(smem + Lay::k), sV = smem_u32(smem + Lay::v);
+      const uint32_t sDS = smem_u32(smem + Lay::ds);
+      bool ok = mbar_wait(&bars->qfull, 0, status, 32);
+      auto grad = [&](int j) -> bool {
+        const int s = j & 1;
+        if (!mbar_wait(&bars->pfull, j & 1, status, 33)) return false;
+        tc_fence_after();
+        const uint32_t kb = sK + s * KV_N * HD * 2;
+#pragma unroll
+        for (int ks = 0; ks < KV_N / 16; ++ks)
+          mma_bf16(tmem + 256, sdesc_sw128(sDS + ks * 32, 16, 1024),
+                   sdesc_sw128(kb + ks * 16 * 128, KV_N * 128, 1024), idG,
+                   (j > 0 || ks > 0) ? 1u : 0u);
+        mma_commit(&bars->dsfree);
+        mma_commit(&bars->kvempty[s]);
+        return true;
+      };
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const int s = j & 1, sb = j & 1;
+        if (!mbar_wait(&bars->kvfull[s], (j >> 1) & 1, status, 34)) { ok = false; break; }
+        if (!mbar_wait(&bars->sfree[sb], ((j >> 1) & 1) ^ 1, status, 35)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t kb = sK + s * KV_N * HD * 2, vb = sV + s * KV_N * HD * 2;
+#pragma unroll
+        for (int ks = 0; ks < HD / 16; ++ks) {
+          const uint32_t qoff = (ks >> 2) * Q_M * 128 + (ks & 3) * 32;
+          const uint32_t koff = (ks >> 2) * KV_N * 128 + (ks & 3) * 32;
+          mma_bf16(tmem + sb * KV_N, sdesc_sw128(sQ + qoff, 16, 1024),
+                   sdesc_sw128(kb + koff, 16, 1024), idS, ks > 0 ? 1u : 0u);
+          mma_bf16(tmem + 128 + sb * KV_N, sdesc_sw128(sO + qoff, 16, 1024),
+                   sdesc_sw128(vb + koff, 16, 1024), idS, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars->sfull[sb]);
+        if (j > 0 && !grad(j - 1)) { ok = false; break; }
+      }
+      if (ok && grad(n_kv - 1)) mma_commit(&bars->done);
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int qrow = qt * Q_M + r;
+    const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+    uint8_t* pDS = smem + Lay::ds;
+    const float c = scale * kLog2e;
+    const float lrow = qrow < S ? __ldg(lse + (int64_t)bh * S + qrow) * kLog2e : INFINITY;
+    const float drow = qrow < S ? __ldg(delta + (int64_t)bh * S + qrow) : 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      const int sb = j & 1;
+      const int k0 = j * KV_N;
+      if (!mbar_wait(&bars->sfull[sb], (j >> 1) & 1, status, 36)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sr[2][32], pr[2][32];
+      tmem_ld32(tmem + lane_addr + sb * KV_N, sr[0]);
+      tmem_ld32(tmem + lane_addr + sb * KV_N + 32, sr[1]);
+      tmem_ld32(tmem + lane_addr + 128 + sb * KV_N, pr[0]);
+      tmem_ld32(tmem + lane_addr + 128 + sb * KV_N + 32, pr[1]);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&bars->sfree[sb]);
+      const bool diag = k0 + KV_N > qt * Q_M;
+      uint32_t dk[KV_N / 2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int col = h * 32 + e;
+          float p0 = ex2(fmaf(__uint_as_float(sr[h][e]), c, -lrow));
+          float p1 = ex2(fmaf(__uint_as_float(sr[h][e + 1]), c, -lrow));
+          if (diag) {
+            p0 = (k0 + col <= qrow) ? p0 : 0.f;
+            p1 = (k0 + col + 1 <= qrow) ? p1 : 0.f;
+          }
+          dk[col >> 1] = pack_bf16x2(p0 * (__uint_as_float(pr[h][e]) - drow),
+                                     p1 * (__uint_as_float(pr[h][e + 1]) - drow));
+        }
+      if (j > 0 && !mbar_wait(&bars->dsfree, (j - 1) & 1, status, 37)) { ok = false; break; }
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc)
+        *reinterpret_cast<uint4*>(pDS + r * 128 + ((cc ^ (r & 7)) << 4)) =
+            make_uint4(dk[cc * 4], dk[cc * 4 + 1], dk[cc * 4 + 2], dk[cc * 4 + 3]);
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars->pfull);
+    }
+    if (ok && mbar_wait(&bars->done, 0, status, 38)) {
+      tc_fence_after();
+      uint4* dst = dqg + ((int64_t)bh * S + qrow) * (HD / 8);
+#pragma unroll
+      for (int cchunk = 0; cchunk < HD / 32; ++cchunk) {
+        uint32_t o[32];
+        tmem_ld32(tmem + lane_addr + 256 + cchunk * 32, o);
+        tmem_ld_wait();
+        if (qrow < S) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(o[v * 8 + 0]) * scale, __uint_as_float(o[v * 8 + 1]) * scale);
+            w.y = pack_bf16x2(__uint_as_float(o[v * 8 + 2]) * scale, __uint_as_float(o[v * 8 + 3]) * scale);
+            w.z = pack_bf16x2(__uint_as_float(o[v * 8 + 4]) * scale, __uint_as_float(o[v * 8 + 5]) * scale);
+            w.w = pack_bf16x2(__uint_as_float(o[v * 8 + 6]) * scale, __uint_as_float(o[v * 8 + 7]) * scale);
+            dst[cchunk * 4 + v] = w;
+          }
+        }
+      }
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Both kernels take one CTA per SM (they allocate 512 TMEM columns).
+constexpr uint32_t kSmemDkdv = DkdvLayout<128>::bytes + 1024;
+constexpr uint32_t kSmemDq = DqLayout<128>::bytes + 1024;
+static_assert(kSmemDkdv <= 232448 && kSmemDq <= 232448, "shared memory");
+static_assert(kSmemDkdv > 232448 / 2 && kSmemDq > 232448 / 2, "one CTA per SM");
+
+template <int HD>
+cudaError_t launch_hd(int BH, int S, float scale, const CUtensorMap* maps_q, const CUtensorMap* maps_kv,
+                      const float* lse, const float* delta, lh_bf16* dqg, lh_bf16* dkg, lh_bf16* dvg,
+                      int* status, cudaStream_t st, int which) {
+  // maps_q: Q, K, V, dO with 64-row boxes (walked tiles of the dK/dV kernel and
+  // K/V of the dQ kernel); maps_kv: the same tensors with 128-row boxes.
+  if (which & 1) {
+    cudaFuncSetAttribute(k_attn_bwd_dkdv<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemDkdv);
+    const int n_kt = (S + KV_M - 1) / KV_M;
+    k_attn_bwd_dkdv<HD><<<n_kt * BH, kThreads, kSmemDkdv, st>>>(
+        maps_q[0], maps_kv[1], maps_kv[2], maps_q[3], lse, delta, (uint4*)dkg, (uint4*)dvg, S, BH,
+        scale, status);
+  }
+  if (which & 2) {
+    cudaFuncSetAttribute(k_attn_bwd_dq<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemDq);
+    const int n_qt = (S + Q_M - 1) / Q_M;
+    k_attn_bwd_dq<HD><<<n_qt * BH, kThreads, kSmemDq, st>>>(maps_kv[0], maps_q[1], maps_q[2],
+                                                           maps_kv[3], lse, delta, (uint4*)dqg, S,
+                                                           BH, scale, status);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool lh_make_tmap_3d(CUtensorMap* m, const void* base, int64_t BH, int64_t rows, int d,
+                     int box_rows);
 
 cudaError_t lh_launch_attn_bwd(int BH, int64_t S, int d, float scale, const lh_bf16* qg,
                                const lh_bf16* kg, const lh_bf16* vg, const lh_bf16* dog,
                                const float* lse, const float* delta, lh_bf16* dqg,
                                lh_bf16* dkg, lh_bf16* dvg, int* status, cudaStream_t st,
-                               int* launches) {
-  return cudaErrorNotSupported;
+                               int which) {
+  CUtensorMap m64[4], m128[4];
+  const lh_bf16* src[4] = {qg, kg, vg, dog};
+  for (int i = 0; i < 4; ++i)
+    if (!lh_make_tmap_3d(&m64[i], src[i], BH, S, d, 64) ||
+        !lh_make_tmap_3d(&m128[i], src[i], BH, S, d, 128))
+      return cudaErrorInvalidValue;
+  if (d == 128)
+    return launch_hd<128>(BH, (int)S, scale, m64, m128, lse, delta, dqg, dkg, dvg, status, st, which);
+  if (d == 64)
+    return launch_hd<64>(BH, (int)S, scale, m64, m128, lse, delta, dqg, dkg, dvg, status, st, which);
+  return cudaErrorInvalidValue;
 }

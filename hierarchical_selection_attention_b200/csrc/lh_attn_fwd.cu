@@ -64,7 +64,8 @@ template <int HD>
 __global__ void __launch_bounds__(kThreads, 1)
     k_attn_fwd(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, uint4* __restrict__ og,
-               float* __restrict__ lse, int S, int BH, float scale_log2, int* status) {
+               uint4* __restrict__ og_lo, float* __restrict__ lse, int S, int BH,
+               float scale_log2, int* status) {
   using Lay = FwdLayout<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -259,15 +260,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem + lane_addr + kColO + c * 32, o);
         tmem_ld_wait();
         if (qrow < S) {
-          uint4* dst = og + ((int64_t)bh * S + qrow) * (HD / 8) + c * 4;
+          const int64_t base = ((int64_t)bh * S + qrow) * (HD / 8) + c * 4;
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(o[v * 8 + 0]) * inv, __uint_as_float(o[v * 8 + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(o[v * 8 + 2]) * inv, __uint_as_float(o[v * 8 + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(o[v * 8 + 4]) * inv, __uint_as_float(o[v * 8 + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(o[v * 8 + 6]) * inv, __uint_as_float(o[v * 8 + 7]) * inv);
-            dst[v] = w;
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(o[v * 8 + e]) * inv;
+            uint4 w, r;
+            w.x = pack_bf16x2(x[0], x[1]); w.y = pack_bf16x2(x[2], x[3]);
+            w.z = pack_bf16x2(x[4], x[5]); w.w = pack_bf16x2(x[6], x[7]);
+            og[base + v] = w;
+            if (og_lo) {
+              const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+              uint32_t rr[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 h = unpack_bf16x2(ww[e]);
+                rr[e] = pack_bf16x2(x[2 * e] - h.x, x[2 * e + 1] - h.y);
+              }
+              r.x = rr[0]; r.y = rr[1]; r.z = rr[2]; r.w = rr[3];
+              og_lo[base + v] = r;
+            }
           }
         }
       }
@@ -314,8 +327,8 @@ bool lh_make_tmap_3d(CUtensorMap* m, const void* base, int64_t BH, int64_t rows,
 }
 
 cudaError_t lh_launch_attn_fwd(int BH, int64_t S, int d, float scale, const lh_bf16* qg,
-                               const lh_bf16* kg, const lh_bf16* vg, lh_bf16* og, float* lse,
-                               int* status, cudaStream_t st) {
+                               const lh_bf16* kg, const lh_bf16* vg, lh_bf16* og,
+                               lh_bf16* og_lo, float* lse, int* status, cudaStream_t st) {
   CUtensorMap tq, tk, tv;
   if (!lh_make_tmap_3d(&tq, qg, BH, S, d, BM) || !lh_make_tmap_3d(&tk, kg, BH, S, d, BN) ||
       !lh_make_tmap_3d(&tv, vg, BH, S, d, BN))
@@ -329,16 +342,16 @@ cudaError_t lh_launch_attn_fwd(int BH, int64_t S, int d, float scale, const lh_b
       cudaFuncSetAttribute(k_attn_fwd<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
       attr = true;
     }
-    k_attn_fwd<128><<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, (uint4*)og, lse, (int)S, BH,
-                                                         scale_log2, status);
+    k_attn_fwd<128><<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, (uint4*)og, (uint4*)og_lo, lse,
+                                                         (int)S, BH, scale_log2, status);
   } else if (d == 64) {
     static bool attr = false;
     if (!attr) {
       cudaFuncSetAttribute(k_attn_fwd<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
       attr = true;
     }
-    k_attn_fwd<64><<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, (uint4*)og, lse, (int)S, BH,
-                                                        scale_log2, status);
+    k_attn_fwd<64><<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, (uint4*)og, (uint4*)og_lo, lse,
+                                                        (int)S, BH, scale_log2, status);
   } else {
     return cudaErrorInvalidValue;
   }

@@ -73,18 +73,20 @@ cudaError_t lh_launch_scatter_atomic(const LhDims& D, const lh_bf16* og,
                                      const int32_t* slot_map, lh_bf16* o, void* ws,
                                      cudaStream_t st, int* launches);
 cudaError_t lh_launch_scatter_bwd(const LhDims& D, const lh_bf16* dout, const lh_bf16* og,
-                                  const int32_t* sel_idx, lh_bf16* dog, float* delta,
-                                  cudaStream_t st);
+                                  const lh_bf16* og_lo, const int32_t* sel_idx, lh_bf16* dog,
+                                  float* delta, cudaStream_t st);
 cudaError_t lh_launch_gather_bwd(const LhDims& D, const lh_bf16* dqg, const lh_bf16* dkg,
                                  const lh_bf16* dvg, const int32_t* slot_map, lh_bf16* dq,
                                  lh_bf16* dk, lh_bf16* dv, cudaStream_t st);
 cudaError_t lh_launch_attn_fwd(int BH, int64_t S, int d, float scale, const lh_bf16* qg,
-                               const lh_bf16* kg, const lh_bf16* vg, lh_bf16* og, float* lse,
-                               int* status, cudaStream_t st);
+                               const lh_bf16* kg, const lh_bf16* vg, lh_bf16* og,
+                               lh_bf16* og_lo, float* lse, int* status, cudaStream_t st);
 cudaError_t lh_launch_attn_delta(int BH, int64_t S, int d, const lh_bf16* og,
-                                 const lh_bf16* dog, float* delta, cudaStream_t st);
+                                 const lh_bf16* og_lo, const lh_bf16* dog, float* delta,
+                                 cudaStream_t st);
+// which: 1 = dK/dV kernel, 2 = dQ kernel, 3 = both.
 cudaError_t lh_launch_attn_bwd(int BH, int64_t S, int d, float scale, const lh_bf16* qg,
                                const lh_bf16* kg, const lh_bf16* vg, const lh_bf16* dog,
                                const float* lse, const float* delta, lh_bf16* dqg,
                                lh_bf16* dkg, lh_bf16* dvg, int* status, cudaStream_t st,
-                               int* launches);
+                               int which);

@@ -151,6 +151,7 @@ __global__ void __launch_bounds__(kThreads) k_scatter_fix2bf16(int64_t n,
 // slot m, vector cv); it sums dO over the shifted range of the slot's entry.
 __global__ void __launch_bounds__(kThreads) k_scatter_bwd(LhDims D, const uint4* __restrict__ dout,
                                                           const uint4* __restrict__ og,
+                                                          const uint4* __restrict__ og_lo,
                                                           const int32_t* __restrict__ sel_idx,
                                                           uint4* __restrict__ dog,
                                                           float* __restrict__ delta) {
@@ -181,10 +182,13 @@ __global__ void __launch_bounds__(kThreads) k_scatter_bwd(LhDims D, const uint4*
   for (; t < stop; ++t) acc8(a, __ldg(src + t * HV));
   const uint4 packed = pack8(a);
   dog[item] = packed;
-  // D from the stored (rounded) values, as the attention backward sees them
+  // D with dO~ as the attention backward sees it (rounded) and the output
+  // to ~16 bits (og + og_lo): D feeds dS = P (dP - D) unscaled, so an error
+  // of one bf16 rounding in O would pass straight into the gradients.
   float rd[8] = {0, 0, 0, 0, 0, 0, 0, 0}, ro[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   acc8(rd, packed);
   acc8(ro, __ldg(og + item));
+  if (og_lo) acc8(ro, __ldg(og_lo + item));
   float s = 0.f;
 #pragma unroll
   for (int e = 0; e < 8; ++e) s = fmaf(rd[e], ro[e], s);
@@ -192,9 +196,10 @@ __global__ void __launch_bounds__(kThreads) k_scatter_bwd(LhDims D, const uint4*
   if (cv == 0) delta[row] = s;
 }
 
-// D = rowsum(dog * og) for the standalone attention backward.
+// D = rowsum(dog * (og + og_lo)) for the standalone attention backward.
 __global__ void __launch_bounds__(kThreads) k_attn_delta(int64_t rows, int V,
                                                          const uint4* __restrict__ og,
+                                                         const uint4* __restrict__ og_lo,
                                                          const uint4* __restrict__ dog,
                                                          float* __restrict__ delta) {
   const int64_t item = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -203,6 +208,7 @@ __global__ void __launch_bounds__(kThreads) k_attn_delta(int64_t rows, int V,
   float rd[8] = {0, 0, 0, 0, 0, 0, 0, 0}, ro[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   acc8(rd, __ldg(dog + item));
   acc8(ro, __ldg(og + item));
+  if (og_lo) acc8(ro, __ldg(og_lo + item));
   float s = 0.f;
 #pragma unroll
   for (int e = 0; e < 8; ++e) s = fmaf(rd[e], ro[e], s);
@@ -289,18 +295,20 @@ cudaError_t lh_launch_scatter_atomic(const LhDims& D, const lh_bf16* og,
 }
 
 cudaError_t lh_launch_scatter_bwd(const LhDims& D, const lh_bf16* dout, const lh_bf16* og,
-                                  const int32_t* sel_idx, lh_bf16* dog, float* delta,
-                                  cudaStream_t st) {
+                                  const lh_bf16* og_lo, const int32_t* sel_idx, lh_bf16* dog,
+                                  float* delta, cudaStream_t st) {
   const int64_t n = (int64_t)D.B * D.H * D.S * (D.d >> 3);
-  k_scatter_bwd<<<nblocks(n), kThreads, 0, st>>>(D, (const uint4*)dout, (const uint4*)og, sel_idx,
-                                                 (uint4*)dog, delta);
+  k_scatter_bwd<<<nblocks(n), kThreads, 0, st>>>(D, (const uint4*)dout, (const uint4*)og,
+                                                 (const uint4*)og_lo, sel_idx, (uint4*)dog, delta);
   return cudaGetLastError();
 }
 
 cudaError_t lh_launch_attn_delta(int BH, int64_t S, int d, const lh_bf16* og,
-                                 const lh_bf16* dog, float* delta, cudaStream_t st) {
+                                 const lh_bf16* og_lo, const lh_bf16* dog, float* delta,
+                                 cudaStream_t st) {
   const int64_t rows = (int64_t)BH * S;
   k_attn_delta<<<nblocks(rows * (d >> 3)), kThreads, 0, st>>>(rows, d >> 3, (const uint4*)og,
+                                                             (const uint4*)og_lo,
                                                              (const uint4*)dog, delta);
   return cudaGetLastError();
 }

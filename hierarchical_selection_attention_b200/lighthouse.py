@@ -56,10 +56,12 @@ def _load():
         "lh_pyramid": (I32, [C, P, P, P, P, P, P, P, P, P]),
         "lh_score_topk": (I32, [C, P, P, P, P, P, SZ, P]),
         "lh_gather": (I32, [C, P, P, P, P, P, P, P, P, P, P, P]),
-        "lh_attn_fwd": (I32, [C, P, P, P, P, P, P]),
-        "lh_attn_bwd": (I32, [C, P, P, P, P, P, P, P, P, P, P, SZ, P]),
+        "lh_attn_fwd": (I32, [C, P, P, P, P, P, P, P]),
+        "lh_attn_bwd": (I32, [C, P, P, P, P, P, P, P, P, P, P, P, SZ, P]),
+        "lh_attn_bwd_dkdv": (I32, [C, P, P, P, P, P, P, P, P, P]),
+        "lh_attn_bwd_dq": (I32, [C, P, P, P, P, P, P, P, P]),
         "lh_scatter": (I32, [C, P, P, P, P, SZ, P]),
-        "lh_scatter_bwd": (I32, [C, P, P, P, P, P, P]),
+        "lh_scatter_bwd": (I32, [C, P, P, P, P, P, P, P]),
         "lh_gather_bwd": (I32, [C, P, P, P, P, P, P, P, P]),
         "lh_forward": (I32, [C, P, P, P, P, P, SZ, P, SZ, P]),
         "lh_backward": (I32, [C, P, SZ, P, P, P, P, P, SZ, P]),
@@ -77,7 +79,7 @@ def _load():
 _lib = _load()
 EXPORTED = ("lh_config_check", "lh_subseq_len", "lh_total_entries", "lh_pooled_rows",
             "lh_workspace_bytes", "lh_saved_offsets", "lh_pyramid", "lh_score_topk", "lh_gather",
-            "lh_attn_fwd", "lh_attn_bwd", "lh_scatter", "lh_scatter_bwd", "lh_gather_bwd",
+            "lh_attn_fwd", "lh_attn_bwd", "lh_attn_bwd_dkdv", "lh_attn_bwd_dq", "lh_scatter", "lh_scatter_bwd", "lh_gather_bwd",
             "lh_forward", "lh_backward", "lh_get_device_status", "lh_status_string",
             "lh_forward_launches", "lh_backward_launches")
 
@@ -139,7 +141,7 @@ def lh_workspace_bytes(cfg: lh_config):
 
 
 def lh_saved_offsets(cfg: lh_config):
-    arr = (ctypes.c_size_t * 7)()
+    arr = (ctypes.c_size_t * 8)()
     _ck(_lib.lh_saved_offsets(ctypes.byref(cfg), arr), "lh_saved_offsets")
     return list(arr)
 
@@ -172,16 +174,30 @@ def lh_gather(cfg, q, k, v, q_lv, k_lv, v_lv, sel_idx, qg, kg, vg, stream=None):
                        _p(kg, BF16), _p(vg, BF16), _stream(stream)), "lh_gather")
 
 
-def lh_attn_fwd(cfg, qg, kg, vg, og, lse, stream=None):
+def lh_attn_fwd(cfg, qg, kg, vg, og, lse, og_lo=None, stream=None):
     _ck(_lib.lh_attn_fwd(ctypes.byref(cfg), _p(qg, BF16), _p(kg, BF16), _p(vg, BF16),
-                         _p(og, BF16), _p(lse, F32), _stream(stream)), "lh_attn_fwd")
+                         _p(og, BF16), _p(og_lo, BF16), _p(lse, F32), _stream(stream)),
+        "lh_attn_fwd")
 
 
-def lh_attn_bwd(cfg, qg, kg, vg, og, lse, dog, dqg, dkg, dvg, ws, stream=None):
+def lh_attn_bwd(cfg, qg, kg, vg, og, lse, dog, dqg, dkg, dvg, ws, og_lo=None, stream=None):
     _ck(_lib.lh_attn_bwd(ctypes.byref(cfg), _p(qg, BF16), _p(kg, BF16), _p(vg, BF16),
-                         _p(og, BF16), _p(lse, F32), _p(dog, BF16), _p(dqg, BF16), _p(dkg, BF16),
+                         _p(og, BF16), _p(og_lo, BF16), _p(lse, F32), _p(dog, BF16),
+                         _p(dqg, BF16), _p(dkg, BF16),
                          _p(dvg, BF16), _p(ws), ws.numel() * ws.element_size(),
                          _stream(stream)), "lh_attn_bwd")
+
+
+def lh_attn_bwd_dkdv(cfg, qg, kg, vg, dog, lse, delta, dkg, dvg, stream=None):
+    _ck(_lib.lh_attn_bwd_dkdv(ctypes.byref(cfg), _p(qg, BF16), _p(kg, BF16), _p(vg, BF16),
+                              _p(dog, BF16), _p(lse, F32), _p(delta, F32), _p(dkg, BF16),
+                              _p(dvg, BF16), _stream(stream)), "lh_attn_bwd_dkdv")
+
+
+def lh_attn_bwd_dq(cfg, qg, kg, vg, dog, lse, delta, dqg, stream=None):
+    _ck(_lib.lh_attn_bwd_dq(ctypes.byref(cfg), _p(qg, BF16), _p(kg, BF16), _p(vg, BF16),
+                            _p(dog, BF16), _p(lse, F32), _p(delta, F32), _p(dqg, BF16),
+                            _stream(stream)), "lh_attn_bwd_dq")
 
 
 def lh_scatter(cfg, og, slot_map, o, ws=None, stream=None):
@@ -190,9 +206,10 @@ def lh_scatter(cfg, og, slot_map, o, ws=None, stream=None):
                         _p(ws), nb, _stream(stream)), "lh_scatter")
 
 
-def lh_scatter_bwd(cfg, dout, og, sel_idx, dog, delta, stream=None):
-    _ck(_lib.lh_scatter_bwd(ctypes.byref(cfg), _p(dout, BF16), _p(og, BF16), _p(sel_idx, I32),
-                            _p(dog, BF16), _p(delta, F32), _stream(stream)), "lh_scatter_bwd")
+def lh_scatter_bwd(cfg, dout, og, sel_idx, dog, delta, og_lo=None, stream=None):
+    _ck(_lib.lh_scatter_bwd(ctypes.byref(cfg), _p(dout, BF16), _p(og, BF16), _p(og_lo, BF16),
+                            _p(sel_idx, I32), _p(dog, BF16), _p(delta, F32), _stream(stream)),
+        "lh_scatter_bwd")
 
 
 def lh_gather_bwd(cfg, dqg, dkg, dvg, slot_map, dq, dk, dv, stream=None):
@@ -243,7 +260,7 @@ def saved_views(cfg: lh_config, saved: torch.Tensor) -> dict:
     return dict(sel_idx=view(0, I32, (B, H, S)), slot_map=view(1, I32, (B, H, P)),
                 qg=view(2, BF16, (B, H, S, d)), kg=view(3, BF16, (B, H, S, d)),
                 vg=view(4, BF16, (B, H, S, d)), og=view(5, BF16, (B, H, S, d)),
-                lse=view(6, F32, (B, H, S)))
+                og_lo=view(6, BF16, (B, H, S, d)), lse=view(7, F32, (B, H, S)))
 
 
 class LighthouseLayer:

@@ -74,7 +74,7 @@ typedef struct {
 } lh_config;
 
 /* Returns LH_OK when the config is valid and supported: B, N, H >= 1,
- * p >= 2, 1 <= L <= 8, p^(L-1) | N, 0 <= (L-1) p k <= sum_{l<L-1} N/p^l,
+ * p >= 2, 1 <= L <= 6, p^(L-1) | N, 0 <= (L-1) p k <= sum_{l<L-1} N/p^l,
  * d in {64, 128}, every index fits in int32 per (b, h). */
 lh_status lh_config_check(const lh_config* cfg);
 
@@ -96,8 +96,8 @@ lh_status lh_workspace_bytes(const lh_config* cfg, size_t* fwd_ws, size_t* bwd_w
                              size_t* saved);
 
 /* Byte offsets inside the saved buffer, in this order: sel_idx (int32
- * [B,H,S]), slot_map (int32 [B,H,P]), qg, kg, vg, og (bf16 [B,H,S,d]),
- * lse (fp32 [B,H,S]).  `offsets` has room for 7 values. */
+ * [B,H,S]), slot_map (int32 [B,H,P]), qg, kg, vg, og, og_lo (bf16
+ * [B,H,S,d]), lse (fp32 [B,H,S]).  `offsets` has room for 8 values. */
 lh_status lh_saved_offsets(const lh_config* cfg, size_t* offsets);
 
 /* (i) + the level-0/coarse scores of (ii), in one pass over Q, K, V.
@@ -138,19 +138,36 @@ lh_status lh_gather(const lh_config* cfg, const lh_bf16* q, const lh_bf16* k,
 /* (iii) causal softmax attention over the gathered sub-sequence (Eq. 9):
  * og[m] = sum_{m' <= m} softmax(scale qg[m].kg[m']) vg[m'], lse[m] = natural
  * log of the softmax normaliser.  tcgen05 tensor cores, fp32 accumulation.
- *  qg, kg, vg in  bf16 [B, H, S, d];  og out bf16 [B, H, S, d];
- *  lse out fp32 [B, H, S]                                                  */
+ *  qg, kg, vg in  bf16 [B, H, S, d];  og out bf16 [B, H, S, d] (the fp32
+ *  result rounded once); og_lo out bf16 [B, H, S, d] or NULL: the rounding
+ *  residual, so og + og_lo carries the output to ~16 significant bits for
+ *  the D = rowsum(dO * O) of the backward;  lse out fp32 [B, H, S]        */
 lh_status lh_attn_fwd(const lh_config* cfg, const lh_bf16* qg, const lh_bf16* kg,
-                      const lh_bf16* vg, lh_bf16* og, float* lse, void* stream);
+                      const lh_bf16* vg, lh_bf16* og, lh_bf16* og_lo, float* lse,
+                      void* stream);
 
-/* Backward of lh_attn_fwd: with P the softmax rows, D = rowsum(dog * og),
- * dS = P (dog vg^T - D): dqg = scale dS kg, dkg = scale dS^T qg,
- * dvg = P^T dog.  Deterministic (no floating-point atomics).
- *  ws scratch of at least bwd_ws bytes.                                    */
+/* Backward of lh_attn_fwd: with P the softmax rows, D = rowsum(dog * O)
+ * (O = og + og_lo; og_lo may be NULL), dS = P (dog vg^T - D):
+ * dqg = scale dS kg, dkg = scale dS^T qg, dvg = P^T dog.  Deterministic (no
+ * floating-point atomics).  Computes D into ws (>= bwd_ws bytes), then runs
+ * lh_attn_bwd_dkdv and lh_attn_bwd_dq. */
 lh_status lh_attn_bwd(const lh_config* cfg, const lh_bf16* qg, const lh_bf16* kg,
-                      const lh_bf16* vg, const lh_bf16* og, const float* lse,
-                      const lh_bf16* dog, lh_bf16* dqg, lh_bf16* dkg, lh_bf16* dvg,
-                      void* ws, size_t ws_bytes, void* stream);
+                      const lh_bf16* vg, const lh_bf16* og, const lh_bf16* og_lo,
+                      const float* lse, const lh_bf16* dog, lh_bf16* dqg, lh_bf16* dkg,
+                      lh_bf16* dvg, void* ws, size_t ws_bytes, void* stream);
+
+/* The dK/dV half of lh_attn_bwd, given delta = D (fp32 [B, H, S], e.g. from
+ * lh_scatter_bwd): one CTA per 128 key rows walks the query rows at and
+ * after its diagonal.  dkg, dvg out bf16 [B, H, S, d]. */
+lh_status lh_attn_bwd_dkdv(const lh_config* cfg, const lh_bf16* qg, const lh_bf16* kg,
+                           const lh_bf16* vg, const lh_bf16* dog, const float* lse,
+                           const float* delta, lh_bf16* dkg, lh_bf16* dvg, void* stream);
+
+/* The dQ half of lh_attn_bwd, given delta: one CTA per 128 query rows walks
+ * the key rows up to its diagonal.  dqg out bf16 [B, H, S, d]. */
+lh_status lh_attn_bwd_dq(const lh_config* cfg, const lh_bf16* qg, const lh_bf16* kg,
+                         const lh_bf16* vg, const lh_bf16* dog, const float* lse,
+                         const float* delta, lh_bf16* dqg, void* stream);
 
 /* (iv) scatter-back, Sec. 3.6: o[t] = sum over levels l of og[slot] for the
  * selected entry (l, i) with (i+1) p^l - 1 <= t <= (i+2) p^l - 2, i.e.
@@ -161,12 +178,14 @@ lh_status lh_scatter(const lh_config* cfg, const lh_bf16* og, const int32_t* slo
                      lh_bf16* o, void* ws, size_t ws_bytes, void* stream);
 
 /* Adjoint of lh_scatter: dog[m] = sum of dO[t] over the shifted range of
- * slot m (clipped to t < N), and delta[m] = rowsum(dog[m] * og[m]) (the D of
- * the attention backward), both per (b, h).
+ * slot m (clipped to t < N), rounded once to bf16, and delta[m] =
+ * rowsum(dog[m] * (og[m] + og_lo[m])) (the D of the attention backward;
+ * og_lo may be NULL), both per (b, h).
  *  dout in bf16 [B, N, H, d]; dog out bf16 [B, H, S, d]; delta out fp32
  *  [B, H, S]                                                               */
 lh_status lh_scatter_bwd(const lh_config* cfg, const lh_bf16* dout, const lh_bf16* og,
-                         const int32_t* sel_idx, lh_bf16* dog, float* delta, void* stream);
+                         const lh_bf16* og_lo, const int32_t* sel_idx, lh_bf16* dog,
+                         float* delta, void* stream);
 
 /* Adjoint of the gather and the mean pooling: dq[t] = sum over levels l of
  * p^-l dqg[slot(l, floor(t/p^l))] for selected entries (unshifted window),
@@ -184,7 +203,8 @@ lh_status lh_forward(const lh_config* cfg, const lh_bf16* q, const lh_bf16* k,
                      void* ws, size_t ws_bytes, void* stream);
 
 /* Whole layer backward from the saved buffer of the matching lh_forward:
- * lh_scatter_bwd, lh_attn_bwd, lh_gather_bwd.  dq, dk, dv out bf16
+ * lh_scatter_bwd (which also gives D), lh_attn_bwd_dkdv, lh_attn_bwd_dq,
+ * lh_gather_bwd.  dq, dk, dv out bf16
  * [B, N, H, d]; `ws` (>= bwd_ws bytes) is scratch.                          */
 lh_status lh_backward(const lh_config* cfg, const void* saved, size_t saved_bytes,
                       const lh_bf16* dout, lh_bf16* dq, lh_bf16* dk, lh_bf16* dv,

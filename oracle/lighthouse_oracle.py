@@ -250,19 +250,22 @@ def attention(qg, kg, vg, scale: float, rows=None, chunk: int = 256):
     return o, lse
 
 
-def attention_bwd(qg, kg, vg, dog, scale: float, chunk: int = 256):
+def attention_bwd(qg, kg, vg, dog, scale: float, chunk: int = 256, rows=None):
     """Gradients of the causal attention with respect to its three inputs.
 
     P = softmax rows, dP = dO V^T, dS = P * (dP - rowsum(P * dP)),
     dQ = scale dS K, dK = scale dS^T Q, dV = P^T dO.
+    ``rows`` restricts the sums over query rows to the given rows (dQ is then
+    exact on those rows, dK and dV hold those rows' share).
     """
     S = qg.shape[0]
     dq = np.zeros_like(qg)
     dk = np.zeros_like(kg)
     dv = np.zeros_like(vg)
     cols = np.arange(S)
-    for a in range(0, S, chunk):
-        r = np.arange(a, min(a + chunk, S))
+    rows = np.arange(S) if rows is None else np.asarray(rows, dtype=np.int64)
+    for a in range(0, rows.shape[0], chunk):
+        r = rows[a:a + chunk]
         s = (qg[r] @ kg.T) * scale
         s[cols[None, :] > r[:, None]] = -np.inf
         mx = s.max(axis=1)

@@ -17,17 +17,21 @@ def f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu", torch.float64).numpy()
 
 
-def close_report(got, want):
+def close_report(got, want, env=None):
+    """(max |x - y| / max(1, env), rel-L2).  env is the magnitude of what was
+    summed to make y (|y| itself by default; for a sum of rounded terms, the
+    sum of the terms' magnitudes, since each term carries its own rounding)."""
     got = np.asarray(got, dtype=np.float64)
     want = np.asarray(want, dtype=np.float64)
+    env = np.abs(want) if env is None else np.asarray(env, dtype=np.float64)
     err = np.abs(got - want)
-    scaled = float(np.max(err / np.maximum(1.0, np.abs(want)))) if err.size else 0.0
+    scaled = float(np.max(err / np.maximum(1.0, env))) if err.size else 0.0
     rel = float(np.linalg.norm(err) / max(np.linalg.norm(want), 1e-30)) if err.size else 0.0
     return scaled, rel
 
 
-def assert_close(got, want, name, max_abs=MAX_ABS, rel_l2=REL_L2):
-    scaled, rel = close_report(got, want)
+def assert_close(got, want, name, max_abs=MAX_ABS, rel_l2=REL_L2, env=None):
+    scaled, rel = close_report(got, want, env)
     assert np.all(np.isfinite(got)), f"{name}: non-finite values"
     assert scaled <= max_abs and rel <= rel_l2, f"{name}: max-abs(scaled) {scaled:.3e}, rel-L2 {rel:.3e}"
     return scaled, rel
@@ -43,3 +47,26 @@ def bf16_ulp(x):
 def head(x: torch.Tensor, b: int, h: int) -> np.ndarray:
     """[B, N, H, d] tensor -> one head's [N, d] fp64 array."""
     return np.ascontiguousarray(x[b, :, h, :].to(torch.float64).cpu().numpy())
+
+
+def attn_bwd_envelopes(qg, kg, vg, dog, scale, chunk=256):
+    """Magnitude envelopes of the attention gradients: the sums that make
+    each gradient with every term replaced by its magnitude.  dS = P dP - P D
+    is formed from two products, so its envelope is P (|dP| + |D|):
+    scale P(|dP|+|D|) |K|, scale (P(|dP|+|D|))^T |Q| and P^T |dO| (fp64)."""
+    S = qg.shape[0]
+    eq, ek, ev = np.zeros_like(qg), np.zeros_like(kg), np.zeros_like(vg)
+    cols = np.arange(S)
+    for a in range(0, S, chunk):
+        r = np.arange(a, min(a + chunk, S))
+        s = (qg[r] @ kg.T) * scale
+        s[cols[None, :] > r[:, None]] = -np.inf
+        pr = np.exp(s - s.max(axis=1)[:, None])
+        pr /= pr.sum(axis=1)[:, None]
+        dp = dog[r] @ vg.T
+        dd = np.abs((pr * dp).sum(axis=1))[:, None]
+        ds = pr * (np.abs(dp) + dd)
+        eq[r] = scale * (ds @ np.abs(kg))
+        ek += scale * (ds.T @ np.abs(qg[r]))
+        ev += pr.T @ np.abs(dog[r])
+    return eq, ek, ev

@@ -52,7 +52,7 @@ def test_sizes_match_oracle(L, B, N, H, d, Lv, p, k):
     assert L.lh_pooled_rows(cfg) == lo.total_entries(N, Lv, p) - N
     fwd, bwd, saved = L.lh_workspace_bytes(cfg)
     S, P = lo.subseq_len(N, Lv, p, k), lo.total_entries(N, Lv, p)
-    assert saved >= B * H * (S * 4 + P * 4 + 4 * S * d * 2 + S * 4)
+    assert saved >= B * H * (S * 4 + P * 4 + 5 * S * d * 2 + S * 4)
     offs = L.lh_saved_offsets(cfg)
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
     assert bwd >= B * H * S * (4 * d * 2 + 4)
