@@ -14,8 +14,7 @@
 //              score row from TMEM, online max / exp2 / row sum, write P as
 //              bf16 into shared memory in the 128-byte-swizzled K-major layout
 //              the next MMA reads, and rescale O in TMEM when the running
-//              max grew by more than 2^8 (otherwise the stale max is kept:
-//              the final division by the row sum makes the result exact).
+//              max of any row of the warp grew.
 // The issuer computes S for tile j+1 while the softmax warps work on tile j
 // and the tensor core runs P V for tile j-1.
 //
@@ -200,8 +199,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float x = __uint_as_float(sr[c][e]);
           if (!diag || col <= r) mx = fmaxf(mx, x);
         }
+      // Exact running max: the row's largest term so far gets p = 1, which
+      // bf16 holds exactly.  (Keeping a stale max, as a lazy-rescale scheme
+      // does, rounds that dominant term by up to 2^-9 and the error reaches
+      // D = rowsum(dO * O) of the backward unscaled.)
       const float m_new = fmaxf(m_used, mx * scale_log2);
-      const bool grow = m_new > m_used + 8.f;
+      const bool grow = m_new > m_used;
       float alpha = 1.f;
       if (grow) {
         alpha = ex2(m_used - m_new);
