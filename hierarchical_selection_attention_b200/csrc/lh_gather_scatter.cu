@@ -75,7 +75,10 @@ __global__ void __launch_bounds__(kThreads) k_gather(LhDims D, const uint4* __re
 }
 
 // (iv) scatter-back, gather side: thread = (b, t, h, vector cv); the entry of
-// level l that reaches t is i = floor((t+1)/p^l) - 1.
+// level l that reaches t is i = floor((t+1)/p^l) - 1.  All slot lookups are
+// issued before any row load, and all row loads before the sum, so a thread
+// waits for two memory round trips rather than two per level.
+template <int L>
 __global__ void __launch_bounds__(kThreads) k_scatter(LhDims D, const uint4* __restrict__ og,
                                                       const int32_t* __restrict__ slot_map,
                                                       uint4* __restrict__ o) {
@@ -91,15 +94,22 @@ __global__ void __launch_bounds__(kThreads) k_scatter(LhDims D, const uint4* __r
   const int b = (int)(bt / D.N);
   const int64_t bh = (int64_t)b * D.H + h;
   const int32_t* sm = slot_map + bh * D.P;
-  float a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  const uint4* src = og + bh * D.S * V + cv;
   const uint32_t t1 = (uint32_t)(t + 1);
-  for (int l = 0; l < D.L; ++l) {
+  int slot[L];
+#pragma unroll
+  for (int l = 0; l < L; ++l) {
     const uint32_t j = t1 / (uint32_t)D.lvl_span[l];
-    if (j == 0) break;
-    const int slot = __ldg(sm + D.lvl_off[l] + j - 1);
-    if (slot < 0) continue;
-    acc8(a, __ldg(og + (bh * D.S + slot) * V + cv));
+    slot[l] = j ? __ldg(sm + D.lvl_off[l] + j - 1) : -1;
   }
+  uint4 row[L];
+#pragma unroll
+  for (int l = 0; l < L; ++l)
+    if (slot[l] >= 0) row[l] = __ldg(src + (int64_t)slot[l] * V);
+  float a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+  for (int l = 0; l < L; ++l)
+    if (slot[l] >= 0) acc8(a, row[l]);
   o[item] = pack8(a);
 }
 
@@ -217,7 +227,9 @@ __global__ void __launch_bounds__(kThreads) k_attn_delta(int64_t rows, int V,
 }
 
 // Adjoint of gather + mean pooling: thread = (b, t, h, vector cv); the level-l
-// entry whose (unshifted) window holds t is i = floor(t / p^l).
+// entry whose (unshifted) window holds t is i = floor(t / p^l).  Slot lookups
+// first, then every row load, then the sums (two memory round trips).
+template <int L>
 __global__ void __launch_bounds__(kThreads) k_gather_bwd(LhDims D, const uint4* __restrict__ dqg,
                                                          const uint4* __restrict__ dkg,
                                                          const uint4* __restrict__ dvg,
@@ -236,17 +248,29 @@ __global__ void __launch_bounds__(kThreads) k_gather_bwd(LhDims D, const uint4* 
   const int b = (int)(bt / D.N);
   const int64_t bh = (int64_t)b * D.H + h;
   const int32_t* sm = slot_map + bh * D.P;
+  int slot[L];
+#pragma unroll
+  for (int l = 0; l < L; ++l)
+    slot[l] = __ldg(sm + D.lvl_off[l] + (uint32_t)t / (uint32_t)D.lvl_span[l]);
+  uint4 rq[L], rk[L], rv[L];
+#pragma unroll
+  for (int l = 0; l < L; ++l) {
+    if (slot[l] >= 0) {
+      const int64_t s = (bh * D.S + slot[l]) * V + cv;
+      rq[l] = __ldg(dqg + s);
+      rk[l] = __ldg(dkg + s);
+      rv[l] = __ldg(dvg + s);
+    }
+  }
   float aq[8] = {0, 0, 0, 0, 0, 0, 0, 0}, ak[8] = {0, 0, 0, 0, 0, 0, 0, 0},
         av[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  for (int l = 0; l < D.L; ++l) {
-    const uint32_t i = (uint32_t)t / (uint32_t)D.lvl_span[l];
-    const int slot = __ldg(sm + D.lvl_off[l] + i);
-    if (slot < 0) continue;
+#pragma unroll
+  for (int l = 0; l < L; ++l) {
+    if (slot[l] < 0) continue;
     const float w = 1.f / (float)D.lvl_span[l];
-    const int64_t s = (bh * D.S + slot) * V + cv;
-    acc8(aq, __ldg(dqg + s), w);
-    acc8(ak, __ldg(dkg + s), w);
-    acc8(av, __ldg(dvg + s), w);
+    acc8(aq, rq[l], w);
+    acc8(ak, rk[l], w);
+    acc8(av, rv[l], w);
   }
   dq[item] = pack8(aq);
   dk[item] = pack8(ak);
@@ -271,7 +295,17 @@ cudaError_t lh_launch_gather(const LhDims& D, const lh_bf16* q, const lh_bf16* k
 cudaError_t lh_launch_scatter(const LhDims& D, const lh_bf16* og, const int32_t* slot_map,
                               lh_bf16* o, cudaStream_t st) {
   const int64_t n = (int64_t)D.B * D.N * D.H * (D.d >> 3);
-  k_scatter<<<nblocks(n), kThreads, 0, st>>>(D, (const uint4*)og, slot_map, (uint4*)o);
+  const unsigned g = nblocks(n);
+  const uint4* x = (const uint4*)og;
+  switch (D.L) {
+    case 1: k_scatter<1><<<g, kThreads, 0, st>>>(D, x, slot_map, (uint4*)o); break;
+    case 2: k_scatter<2><<<g, kThreads, 0, st>>>(D, x, slot_map, (uint4*)o); break;
+    case 3: k_scatter<3><<<g, kThreads, 0, st>>>(D, x, slot_map, (uint4*)o); break;
+    case 4: k_scatter<4><<<g, kThreads, 0, st>>>(D, x, slot_map, (uint4*)o); break;
+    case 5: k_scatter<5><<<g, kThreads, 0, st>>>(D, x, slot_map, (uint4*)o); break;
+    case 6: k_scatter<6><<<g, kThreads, 0, st>>>(D, x, slot_map, (uint4*)o); break;
+    default: return cudaErrorInvalidValue;
+  }
   return cudaGetLastError();
 }
 
@@ -317,8 +351,17 @@ cudaError_t lh_launch_gather_bwd(const LhDims& D, const lh_bf16* dqg, const lh_b
                                  const lh_bf16* dvg, const int32_t* slot_map, lh_bf16* dq,
                                  lh_bf16* dk, lh_bf16* dv, cudaStream_t st) {
   const int64_t n = (int64_t)D.B * D.N * D.H * (D.d >> 3);
-  k_gather_bwd<<<nblocks(n), kThreads, 0, st>>>(D, (const uint4*)dqg, (const uint4*)dkg,
-                                                (const uint4*)dvg, slot_map, (uint4*)dq,
-                                                (uint4*)dk, (uint4*)dv);
+  const unsigned g = nblocks(n);
+  const uint4 *a = (const uint4*)dqg, *b = (const uint4*)dkg, *c = (const uint4*)dvg;
+  uint4 *x = (uint4*)dq, *y = (uint4*)dk, *z = (uint4*)dv;
+  switch (D.L) {
+    case 1: k_gather_bwd<1><<<g, kThreads, 0, st>>>(D, a, b, c, slot_map, x, y, z); break;
+    case 2: k_gather_bwd<2><<<g, kThreads, 0, st>>>(D, a, b, c, slot_map, x, y, z); break;
+    case 3: k_gather_bwd<3><<<g, kThreads, 0, st>>>(D, a, b, c, slot_map, x, y, z); break;
+    case 4: k_gather_bwd<4><<<g, kThreads, 0, st>>>(D, a, b, c, slot_map, x, y, z); break;
+    case 5: k_gather_bwd<5><<<g, kThreads, 0, st>>>(D, a, b, c, slot_map, x, y, z); break;
+    case 6: k_gather_bwd<6><<<g, kThreads, 0, st>>>(D, a, b, c, slot_map, x, y, z); break;
+    default: return cudaErrorInvalidValue;
+  }
   return cudaGetLastError();
 }
