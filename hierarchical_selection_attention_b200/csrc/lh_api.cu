@@ -423,6 +423,46 @@ const char* lh_status_string(lh_status s) {
   return "unknown status";
 }
 
+// ---------------------------------------------------------------------------
+// lh_score_topk without a caller workspace.  The selection scratch (digit
+// histograms, per-head threshold state, per-block counts) lives in this
+// fixed device array instead; every device that loads the library keeps it
+// until the process exits.  Host code must not hand the array's name to a
+// kernel (on the host it names a stand-in, not device memory): the device
+// address is looked up once per device with cudaGetSymbolAddress and that
+// pointer is what the kernels get.
+constexpr size_t kNoAllocScratchBytes = (size_t)8 << 20;  // 8 MiB
+static __device__ __align__(256) unsigned char g_topk_scratch[kNoAllocScratchBytes];
+
+static void* topk_scratch_ptr() {
+  static void* ptrs[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_topk_scratch) != cudaSuccess || p == nullptr) return nullptr;
+    ptrs[dev] = p;
+  }
+  return ptrs[dev];
+}
+
+lh_status lh_score_topk_noalloc(const lh_config* cfg, const float* qk, const float* kq,
+                                int32_t* sel_idx, int32_t* slot_map, void* stream) {
+  LH_TRY(check(cfg));
+  if (!all_aligned(qk, kq, sel_idx, slot_map)) return LH_ERR_INVALID_ARGUMENT;
+  const LhDims D = launch_dims(cfg);
+  if (!D.status) return LH_ERR_CUDA;
+  if (lh_select_ws_bytes(D) > kNoAllocScratchBytes) return LH_ERR_WORKSPACE;
+  void* scratch = topk_scratch_ptr();
+  if (!scratch) return LH_ERR_CUDA;
+  // lh_launch_select zeroes the histograms it accumulates into before use;
+  // the state and block counts are written before they are read.
+  return cu(lh_launch_select(D, qk, kq, sel_idx, slot_map, scratch, (cudaStream_t)stream,
+                             nullptr));
+}
+
+size_t lh_score_topk_noalloc_max_bytes(void) { return kNoAllocScratchBytes; }
+
 int32_t lh_forward_launches(const lh_config* cfg) {
   if (check(cfg) != LH_OK) return -1;
   const LhDims D = dims(cfg);

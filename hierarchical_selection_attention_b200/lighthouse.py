@@ -55,6 +55,8 @@ def _load():
         "lh_saved_offsets": (I32, [C, ctypes.POINTER(SZ)]),
         "lh_pyramid": (I32, [C, P, P, P, P, P, P, P, P, P]),
         "lh_score_topk": (I32, [C, P, P, P, P, P, SZ, P]),
+        "lh_score_topk_noalloc": (I32, [C, P, P, P, P, P]),
+        "lh_score_topk_noalloc_max_bytes": (SZ, []),
         "lh_gather": (I32, [C, P, P, P, P, P, P, P, P, P, P, P]),
         "lh_attn_fwd": (I32, [C, P, P, P, P, P, P, P]),
         "lh_attn_bwd": (I32, [C, P, P, P, P, P, P, P, P, P, P, P, SZ, P]),
@@ -78,7 +80,8 @@ def _load():
 
 _lib = _load()
 EXPORTED = ("lh_config_check", "lh_subseq_len", "lh_total_entries", "lh_pooled_rows",
-            "lh_workspace_bytes", "lh_saved_offsets", "lh_pyramid", "lh_score_topk", "lh_gather",
+            "lh_workspace_bytes", "lh_saved_offsets", "lh_pyramid", "lh_score_topk",
+            "lh_score_topk_noalloc", "lh_score_topk_noalloc_max_bytes", "lh_gather",
             "lh_attn_fwd", "lh_attn_bwd", "lh_attn_bwd_dkdv", "lh_attn_bwd_dq", "lh_scatter", "lh_scatter_bwd", "lh_gather_bwd",
             "lh_forward", "lh_backward", "lh_get_device_status", "lh_status_string",
             "lh_forward_launches", "lh_backward_launches")
@@ -166,6 +169,19 @@ def lh_score_topk(cfg, qk, kq, sel_idx, slot_map, ws, stream=None):
     _ck(_lib.lh_score_topk(ctypes.byref(cfg), _p(qk, F32), _p(kq, F32), _p(sel_idx, I32),
                            _p(slot_map, I32), _p(ws), ws.numel() * ws.element_size(),
                            _stream(stream)), "lh_score_topk")
+
+
+def lh_score_topk_noalloc(cfg, qk, kq, sel_idx, slot_map, stream=None):
+    """lh_score_topk without a workspace argument: the scratch is the library's
+    own fixed device array (see the header for the size limit and the rule
+    that calls on one device must not overlap)."""
+    _ck(_lib.lh_score_topk_noalloc(ctypes.byref(cfg), _p(qk, F32), _p(kq, F32),
+                                   _p(sel_idx, I32), _p(slot_map, I32), _stream(stream)),
+        "lh_score_topk_noalloc")
+
+
+def lh_score_topk_noalloc_max_bytes() -> int:
+    return _lib.lh_score_topk_noalloc_max_bytes()
 
 
 def lh_gather(cfg, q, k, v, q_lv, k_lv, v_lv, sel_idx, qg, kg, vg, stream=None):

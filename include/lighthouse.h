@@ -127,6 +127,32 @@ lh_status lh_score_topk(const lh_config* cfg, const float* qk, const float* kq,
                         int32_t* sel_idx, int32_t* slot_map, void* ws, size_t ws_bytes,
                         void* stream);
 
+/* lh_score_topk for callers that cannot allocate device memory.  The paper
+ * has no counterpart: this is a convenience of this library.  Some callers
+ * cannot hand the library a workspace: their device memory is owned by
+ * another allocator that must not be bypassed, their plugin interface has no
+ * slot for a scratch pointer, or their step may not allocate at all.  This
+ * entry point needs none: its scratch is a fixed 8 MiB device array inside
+ * the library (lh_score_topk_noalloc_max_bytes), held by every device that
+ * loads the library until the process exits.  It allocates nothing and
+ * calls no allocating routine.
+ *  - Same arguments and results as lh_score_topk, minus ws / ws_bytes.
+ *  - Returns LH_ERR_WORKSPACE when the selection scratch of cfg (the fwd_ws
+ *    part that lh_score_topk uses) exceeds the array; roughly B*H*50 KB +
+ *    B*H*N/256 bytes, so B*H <= 128 fits at N = 2^20.
+ *  - The first call on a device looks up the array's device address (once
+ *    per device, with that device current); make that first call before any
+ *    stream capture.
+ *  - Every call on a device shares the one array and leaves its contents
+ *    behind; each call clears what it needs zeroed.  Calls whose work
+ *    overlaps on the GPU (different streams, no ordering between them) race
+ *    on the array: order them, e.g. on one stream. */
+lh_status lh_score_topk_noalloc(const lh_config* cfg, const float* qk, const float* kq,
+                                int32_t* sel_idx, int32_t* slot_map, void* stream);
+
+/* Size in bytes of the fixed scratch array of lh_score_topk_noalloc. */
+size_t lh_score_topk_noalloc_max_bytes(void);
+
 /* (iii) gather: row m of qg/kg/vg is the pyramid entry sel_idx[m]
  * (level 0 from q/k/v, coarser levels from q_lv/k_lv/v_lv).
  *  qg, kg, vg out bf16 [B, H, S, d]                                        */
