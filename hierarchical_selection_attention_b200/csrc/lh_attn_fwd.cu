@@ -4,24 +4,27 @@
 // the mask is the plain S x S causal one, so this is a causal attention
 // forward on [BH, S, d] bf16 tensors, written for the sm_100a tensor cores.
 //
-// One CTA owns a tile of 128 query rows of one (b, h) and walks the key/value
-// tiles of 128 rows up to the diagonal.  Warp roles:
-//   warp 0     TMA producer: Q once, then K and V tiles into a 2-stage ring;
-//   warp 1     tcgen05 issuer (one thread): S = Q K^T into one of two TMEM
-//              score buffers, then O += P V into the TMEM accumulator; each
-//              group is committed to an mbarrier;
-//   warps 2-5  softmax, one query row per thread (TMEM lane = row): read the
-//              score row from TMEM, online max / exp2 / row sum, write P as
-//              bf16 into shared memory in the 128-byte-swizzled K-major layout
-//              the next MMA reads, and rescale O in TMEM when the running
-//              max of any row of the warp grew.
-// The issuer computes S for tile j+1 while the softmax warps work on tile j
-// and the tensor core runs P V for tile j-1.
+// One CTA owns two tiles of 128 query rows of one (b, h), A and B (rows
+// 256 g .. 256 g + 255), and walks the key/value tiles of 128 rows up to B's
+// diagonal (A skips the last one).  Warp roles:
+//   warp 0      TMA producer: Q_A and Q_B once, then K and V tiles into a
+//               2-stage ring;
+//   warp 1      tcgen05 issuer (one thread).  Per key tile j it issues
+//               S_A = Q_A K^T, S_B = Q_B K^T into TMEM, then, as each softmax
+//               warpgroup hands back its P, O_X += P_X V with P_X read from
+//               TMEM (A operand in tensor memory) and V from shared memory;
+//   warps 2-5   softmax of tile A, warps 6-9 softmax of tile B: one query
+//               row per thread (TMEM lane = row).  Each reads its score row,
+//               keeps the exact running max and the row sum, writes
+//               P = exp2(s - max) as bf16 pairs over the score columns it
+//               has just read, and rescales O_X in TMEM when a row's max grew.
+// While warpgroup A turns S_A into P_A, the tensor core works on S_B or on
+// P_B V, and the other way round.
 //
-// TMEM: two 128-column fp32 score buffers and a d-column fp32 accumulator
-// (512 columns allocated, one CTA per SM).  Shared memory: Q (128 x d), two
-// K and two V stages (128 x d each) and P (128 x 128), all bf16, 128-byte
-// swizzled, 1024-byte aligned.
+// TMEM (512 columns, one CTA per SM): S_A 0..127, S_B 128..255 (P_X packed
+// into the first 64 columns of S_X), O_A and O_B (d columns each) from 256.
+// Shared memory: Q_A, Q_B, two K and two V stages (128 x d bf16 each),
+// 128-byte swizzled, 1024-byte aligned.
 #include <cudaTypedefs.h>
 
 #include "lh_sm100.cuh"
@@ -33,29 +36,27 @@ using namespace sm100;
 constexpr int BM = 128;
 constexpr int BN = 128;
 constexpr int NST = 2;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;    // two score buffers: columns 0 and 128
-constexpr uint32_t kColO = 256;  // accumulator
 
 template <int HD>
 struct FwdLayout {
-  static constexpr uint32_t q = 0;
-  static constexpr uint32_t k = q + BM * HD * 2;
+  static constexpr uint32_t q = 0;                       // Q_A, Q_B
+  static constexpr uint32_t k = q + 2 * BM * HD * 2;
   static constexpr uint32_t v = k + NST * BN * HD * 2;
-  static constexpr uint32_t p = v + NST * BN * HD * 2;
-  static constexpr uint32_t bar = p + BM * BN * 2;
+  static constexpr uint32_t bar = v + NST * BN * HD * 2;
   static constexpr uint32_t bytes = bar + 256;
 };
 
-// Force one CTA per SM (TMEM is allocated at 512 columns).
+// At least half the shared memory of an SM: one CTA per SM, since each
+// allocates all 512 TMEM columns.
 constexpr uint32_t kSmemBytes = FwdLayout<128>::bytes + 1024;
+static_assert(kSmemBytes > 232448 / 2 && kSmemBytes <= 232448, "one CTA per SM");
 
 struct Bars {
   uint64_t qfull;
   uint64_t kfull[NST], kempty[NST], vfull[NST], vempty[NST];
-  uint64_t sfull[2], sfree[2];
-  uint64_t pfull, pvdone;
+  uint64_t sfull[2], pfull[2], odone[2];
   uint32_t tmem_base;
 };
 
@@ -73,15 +74,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sQ = smem_u32(smem + Lay::q);
   const uint32_t sK = smem_u32(smem + Lay::k);
   const uint32_t sV = smem_u32(smem + Lay::v);
-  uint8_t* pP = smem + Lay::p;
-  const uint32_t sP = smem_u32(pP);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n_qt = (S + BM - 1) / BM;
-  const int qt = n_qt - 1 - (int)(blockIdx.x / BH);  // longest rows first
+  const int n_pair = (n_qt + 1) / 2;
+  const int g = n_pair - 1 - (int)(blockIdx.x / BH);  // longest rows first
   const int bh = (int)(blockIdx.x % BH);
-  const int n_kv = qt + 1;
+  const int qt_a = 2 * g, qt_b = 2 * g + 1;
+  const int n_a = qt_a + 1;                           // key tiles of tile A
+  const int n_b = qt_b < n_qt ? qt_b + 1 : 0;         // 0: tile B is past the end
+  const int n_kv = n_b ? n_b : n_a;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->qfull, 1);
@@ -91,12 +94,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->vfull[s], 1);
       mbar_init(&bars->vempty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars->sfull[s], 1);
-      mbar_init(&bars->sfree[s], 128);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bars->sfull[x], 1);
+      mbar_init(&bars->pfull[x], 128);
+      mbar_init(&bars->odone[x], 1);
     }
-    mbar_init(&bars->pfull, 128);
-    mbar_init(&bars->pvdone, 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -113,9 +115,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_expect_tx(&bars->qfull, BM * HD * 2);
-      for (int blk = 0; blk < HD / 64; ++blk)
-        tma_load_3d(&tmQ, &bars->qfull, smem + Lay::q + blk * BM * 128, 64 * blk, qt * BM, bh);
+      mbar_expect_tx(&bars->qfull, 2 * BM * HD * 2);
+      for (int x = 0; x < 2; ++x)
+        for (int blk = 0; blk < HD / 64; ++blk)
+          tma_load_3d(&tmQ, &bars->qfull, smem + Lay::q + x * BM * HD * 2 + blk * BM * 128,
+                      64 * blk, (qt_a + x) * BM, bh);
       for (int j = 0; j < n_kv; ++j) {
         const int s = j % NST;
         const uint32_t ph = (j / NST) & 1;
@@ -136,153 +140,150 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idS = idesc_bf16(BM, BN, 0, 0);
       constexpr uint32_t idO = idesc_bf16(BM, HD, 0, 1);
       bool ok = mbar_wait(&bars->qfull, 0, status, 3);
-      auto pv = [&](int i) -> bool {
-        const int s = i % NST;
-        if (!mbar_wait(&bars->pfull, i & 1, status, 4)) return false;
-        if (!mbar_wait(&bars->vfull[s], (i / NST) & 1, status, 5)) return false;
-        tc_fence_after();
-        const uint32_t vb = sV + s * BN * HD * 2;
-#pragma unroll
-        for (int ks = 0; ks < BN / 16; ++ks) {
-          const uint64_t a = sdesc_sw128(sP + (ks >> 2) * BM * 128 + (ks & 3) * 32, 16, 1024);
-          const uint64_t b = sdesc_sw128(vb + ks * 16 * 128, BN * 128, 1024);
-          mma_bf16(tmem + kColO, a, b, idO, (i > 0 || ks > 0) ? 1u : 0u);
-        }
-        mma_commit(&bars->pvdone);
-        mma_commit(&bars->vempty[s]);
-        return true;
-      };
       for (int j = 0; ok && j < n_kv; ++j) {
         const int s = j % NST;
-        const int sb = j & 1;
-        if (!mbar_wait(&bars->kfull[s], (j / NST) & 1, status, 6)) { ok = false; break; }
-        if (!mbar_wait(&bars->sfree[sb], ((j >> 1) & 1) ^ 1, status, 7)) { ok = false; break; }
-        tc_fence_after();
+        const uint32_t ph = (j / NST) & 1;
+        if (!mbar_wait(&bars->kfull[s], ph, status, 4)) { ok = false; break; }
         const uint32_t kb = sK + s * BN * HD * 2;
+        for (int x = 0; x < 2 && ok; ++x) {
+          if (j >= (x ? n_b : n_a)) continue;
+          // S_X shares its columns with P_X of the last tile: P_X V must be done
+          if (j > 0 && !mbar_wait(&bars->odone[x], (j - 1) & 1, status, 5)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t qb = sQ + x * BM * HD * 2;
 #pragma unroll
-        for (int ks = 0; ks < HD / 16; ++ks) {
-          const uint64_t a = sdesc_sw128(sQ + (ks >> 2) * BM * 128 + (ks & 3) * 32, 16, 1024);
-          const uint64_t b = sdesc_sw128(kb + (ks >> 2) * BN * 128 + (ks & 3) * 32, 16, 1024);
-          mma_bf16(tmem + kColS + sb * BN, a, b, idS, ks > 0 ? 1u : 0u);
+          for (int ks = 0; ks < HD / 16; ++ks) {
+            const uint64_t a = sdesc_sw128(qb + (ks >> 2) * BM * 128 + (ks & 3) * 32, 16, 1024);
+            const uint64_t b = sdesc_sw128(kb + (ks >> 2) * BN * 128 + (ks & 3) * 32, 16, 1024);
+            mma_bf16(tmem + x * 128, a, b, idS, ks > 0 ? 1u : 0u);
+          }
+          mma_commit(&bars->sfull[x]);
         }
-        mma_commit(&bars->sfull[sb]);
+        if (!ok) break;
         mma_commit(&bars->kempty[s]);
-        if (j > 0 && !pv(j - 1)) { ok = false; break; }
+        if (!mbar_wait(&bars->vfull[s], ph, status, 6)) { ok = false; break; }
+        const uint32_t vb = sV + s * BN * HD * 2;
+        for (int x = 0; x < 2 && ok; ++x) {
+          if (j >= (x ? n_b : n_a)) continue;
+          if (!mbar_wait(&bars->pfull[x], j & 1, status, 7)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int ks = 0; ks < BN / 16; ++ks) {
+            const uint64_t b = sdesc_sw128(vb + ks * 16 * 128, BN * 128, 1024);
+            mma_bf16_ts(tmem + 256 + x * HD, tmem + x * 128 + ks * 8, b, idO,
+                        (j > 0 || ks > 0) ? 1u : 0u);
+          }
+          mma_commit(&bars->odone[x]);
+        }
+        if (!ok) break;
+        mma_commit(&bars->vempty[s]);
       }
-      if (ok) pv(n_kv - 1);
     }
   } else {
-    // softmax warps: TMEM lane quarter = warp % 4
+    // softmax warpgroup x: warps 2-5 (x = 0) and 6-9 (x = 1)
+    const int x = (warp - 2) >> 2;
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;       // row in the tile
+    const int r = quarter * 32 + lane;       // row in the tile = TMEM lane
+    const int qt = qt_a + x;
     const int qrow = qt * BM + r;            // row in the sequence
+    const int n_x = x ? n_b : n_a;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_addr + x * 128;
+    const uint32_t tO = tmem + lane_addr + 256 + x * HD;
     float m_used = -INFINITY, lsum = 0.f;
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      const int sb = j & 1;
-      if (!mbar_wait(&bars->sfull[sb], (j >> 1) & 1, status, 8)) { ok = false; break; }
+    for (int j = 0; j < n_x; ++j) {
+      if (!mbar_wait(&bars->sfull[x], j & 1, status, 8)) { ok = false; break; }
       tc_fence_after();
       uint32_t sr[BN / 32][32];
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) tmem_ld32(tmem + lane_addr + kColS + sb * BN + c * 32, sr[c]);
+      for (int c = 0; c < BN / 32; ++c) tmem_ld32(tS + c * 32, sr[c]);
       tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&bars->sfree[sb]);
       const bool diag = (j == qt);
       float mx = -INFINITY;
+      if (diag) {
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c)
+        for (int c = 0; c < BN / 32; ++c)
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int col = c * 32 + e;
-          const float x = __uint_as_float(sr[c][e]);
-          if (!diag || col <= r) mx = fmaxf(mx, x);
-        }
+          for (int e = 0; e < 32; ++e)
+            if (c * 32 + e <= r) mx = fmaxf(mx, __uint_as_float(sr[c][e]));
+      } else {
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[c][e]));
+      }
       // Exact running max: the row's largest term so far gets p = 1, which
-      // bf16 holds exactly.  (Keeping a stale max, as a lazy-rescale scheme
-      // does, rounds that dominant term by up to 2^-9 and the error reaches
+      // bf16 holds exactly.  (A stale max, as lazy rescaling keeps, would
+      // round that dominant term by up to 2^-9, and the error would reach
       // D = rowsum(dO * O) of the backward unscaled.)
       const float m_new = fmaxf(m_used, mx * scale_log2);
       const bool grow = m_new > m_used;
-      float alpha = 1.f;
-      if (grow) {
-        alpha = ex2(m_used - m_new);
-        m_used = m_new;
-      }
+      const float alpha = grow ? ex2(m_used - m_new) : 1.f;
+      m_used = m_new;
       float rs = 0.f;
-      uint32_t pk[BN / 2];
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c)
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const int col = c * 32 + e;
           float p0 = ex2(fmaf(__uint_as_float(sr[c][e]), scale_log2, -m_used));
           float p1 = ex2(fmaf(__uint_as_float(sr[c][e + 1]), scale_log2, -m_used));
           if (diag) {
-            p0 = col <= r ? p0 : 0.f;
-            p1 = col + 1 <= r ? p1 : 0.f;
+            p0 = (c * 32 + e <= r) ? p0 : 0.f;
+            p1 = (c * 32 + e + 1 <= r) ? p1 : 0.f;
           }
           rs += p0 + p1;
-          pk[col >> 1] = pack_bf16x2(p0, p1);
+          pk[e >> 1] = pack_bf16x2(p0, p1);
         }
-      lsum = lsum * alpha + rs;
-      if (j > 0 && !mbar_wait(&bars->pvdone, (j - 1) & 1, status, 9)) { ok = false; break; }
-      // P into the swizzled K-major layout: 16-byte chunk cc of row r at
-      // block (col / 64), chunk (cc ^ (r % 8)).
-#pragma unroll
-      for (int q = 0; q < BN / 8; ++q) {
-        const int blk = q >> 3, cc = q & 7;
-        uint4 w;
-        w.x = pk[q * 4 + 0]; w.y = pk[q * 4 + 1]; w.z = pk[q * 4 + 2]; w.w = pk[q * 4 + 3];
-        *reinterpret_cast<uint4*>(pP + blk * BM * 128 + r * 128 + ((cc ^ (r & 7)) << 4)) = w;
+        tmem_st16(tS + c * 16, pk);  // P over the score columns already read
       }
+      lsum = lsum * alpha + rs;
+      // O_X holds P V of the earlier tiles (P_X V of tile j-1 finished before
+      // S_X of tile j was issued); bring it to the new max.
       if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        tc_fence_after();
 #pragma unroll
         for (int c = 0; c < HD / 32; ++c) {
           uint32_t o[32];
-          tmem_ld32(tmem + lane_addr + kColO + c * 32, o);
+          tmem_ld32(tO + c * 32, o);
           tmem_ld_wait();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(tmem + lane_addr + kColO + c * 32, o);
+          tmem_st32(tO + c * 32, o);
         }
-        tmem_st_wait();
       }
-      fence_async_smem();
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bars->pfull);
+      mbar_arrive(&bars->pfull[x]);
     }
-    if (ok && mbar_wait(&bars->pvdone, (n_kv - 1) & 1, status, 10)) {
+    if (ok && n_x > 0 && mbar_wait(&bars->odone[x], (n_x - 1) & 1, status, 10)) {
       tc_fence_after();
       const float inv = 1.f / lsum;
 #pragma unroll
       for (int c = 0; c < HD / 32; ++c) {
         uint32_t o[32];
-        tmem_ld32(tmem + lane_addr + kColO + c * 32, o);
+        tmem_ld32(tO + c * 32, o);
         tmem_ld_wait();
         if (qrow < S) {
           const int64_t base = ((int64_t)bh * S + qrow) * (HD / 8) + c * 4;
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
-            float x[8];
+            float xv[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(o[v * 8 + e]) * inv;
-            uint4 w, r;
-            w.x = pack_bf16x2(x[0], x[1]); w.y = pack_bf16x2(x[2], x[3]);
-            w.z = pack_bf16x2(x[4], x[5]); w.w = pack_bf16x2(x[6], x[7]);
+            for (int e = 0; e < 8; ++e) xv[e] = __uint_as_float(o[v * 8 + e]) * inv;
+            uint4 w;
+            w.x = pack_bf16x2(xv[0], xv[1]); w.y = pack_bf16x2(xv[2], xv[3]);
+            w.z = pack_bf16x2(xv[4], xv[5]); w.w = pack_bf16x2(xv[6], xv[7]);
             og[base + v] = w;
             if (og_lo) {
               const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
               uint32_t rr[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
-                const float2 h = unpack_bf16x2(ww[e]);
-                rr[e] = pack_bf16x2(x[2 * e] - h.x, x[2 * e + 1] - h.y);
+                const float2 hh = unpack_bf16x2(ww[e]);
+                rr[e] = pack_bf16x2(xv[2 * e] - hh.x, xv[2 * e + 1] - hh.y);
               }
-              r.x = rr[0]; r.y = rr[1]; r.z = rr[2]; r.w = rr[3];
-              og_lo[base + v] = r;
+              og_lo[base + v] = make_uint4(rr[0], rr[1], rr[2], rr[3]);
             }
           }
         }
@@ -337,22 +338,14 @@ cudaError_t lh_launch_attn_fwd(int BH, int64_t S, int d, float scale, const lh_b
       !lh_make_tmap_3d(&tv, vg, BH, S, d, BN))
     return cudaErrorInvalidValue;
   const int n_qt = (int)((S + BM - 1) / BM);
-  const dim3 grid((unsigned)(n_qt * BH));
+  const dim3 grid((unsigned)(((n_qt + 1) / 2) * BH));
   const float scale_log2 = scale * 1.4426950408889634f;
   if (d == 128) {
-    static bool attr = false;
-    if (!attr) {
-      cudaFuncSetAttribute(k_attn_fwd<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-      attr = true;
-    }
+    cudaFuncSetAttribute(k_attn_fwd<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     k_attn_fwd<128><<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, (uint4*)og, (uint4*)og_lo, lse,
                                                          (int)S, BH, scale_log2, status);
   } else if (d == 64) {
-    static bool attr = false;
-    if (!attr) {
-      cudaFuncSetAttribute(k_attn_fwd<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-      attr = true;
-    }
+    cudaFuncSetAttribute(k_attn_fwd<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     k_attn_fwd<64><<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, (uint4*)og, (uint4*)og_lo, lse,
                                                         (int)S, BH, scale_log2, status);
   } else {
