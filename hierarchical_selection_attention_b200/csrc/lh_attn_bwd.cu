@@ -15,11 +15,14 @@
 //                   rows up to its diagonal, recomputing S and dP, and
 //                   accumulates dQ in TMEM.
 //
-// Warp roles as in the forward: warp 0 issues TMA loads (2-stage ring of the
-// walked tiles), warp 1 issues the MMAs from one thread and commits them to
-// mbarriers, warps 2-5 own one TMEM lane (= one row of the stationary tile)
-// each, turn scores into P and dS in fp32, and write them to shared memory
-// as bf16 in the 128-byte-swizzled K-major layout the gradient MMAs read.
+// Warp roles: warp 0 issues TMA loads (2-stage ring of the walked tiles),
+// warp 1 issues the MMAs from one thread and commits them to mbarriers, and
+// two softmax warpgroups (warps 2-9) own the TMEM lanes (= the rows of the
+// stationary tile), each warpgroup half of the walked tile's columns: they
+// turn scores into P and dS in fp32 and write them to shared memory as bf16
+// in the 128-byte-swizzled K-major layout the gradient MMAs read.  (The
+// backward softmax is elementwise given LSE and D, so the two halves need no
+// exchange; two warps per SM sub-partition hide each other's latency.)
 // The same shared-memory tile of Q, dO or K serves as a K-major operand in
 // one MMA and as an MN-major operand in another.
 #include "lh_sm100.cuh"
@@ -28,7 +31,10 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 192;
+// warp 0 TMA, warp 1 MMA, warps 2-9 two softmax warpgroups: warp w owns TMEM
+// lanes 32 (w % 4) .. +31 and half (w - 2) / 4 of the walked tile's columns.
+constexpr int kThreads = 320;
+constexpr int kSoftmax = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -37,21 +43,22 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int KV_M = 128;  // stationary key rows
 constexpr int Q_N = 64;    // walked query rows per tile
 
+constexpr int QST = 3;     // stages of the walked Q / dO ring
+
 template <int HD>
 struct DkdvLayout {
   static constexpr uint32_t k = 0;
   static constexpr uint32_t v = k + KV_M * HD * 2;
-  static constexpr uint32_t q = v + KV_M * HD * 2;            // 2 stages
-  static constexpr uint32_t dO = q + 2 * Q_N * HD * 2;        // 2 stages
-  static constexpr uint32_t p = dO + 2 * Q_N * HD * 2;        // [128][64] bf16
-  static constexpr uint32_t ds = p + KV_M * Q_N * 2;          // [128][64] bf16
-  static constexpr uint32_t vec = ds + KV_M * Q_N * 2;        // lse/delta, 2 x 2 x 64 fp32
-  static constexpr uint32_t bar = vec + 4 * Q_N * 4;
+  static constexpr uint32_t q = v + KV_M * HD * 2;            // QST stages
+  static constexpr uint32_t dO = q + QST * Q_N * HD * 2;      // QST stages
+  static constexpr uint32_t p = dO + QST * Q_N * HD * 2;      // 2 x [128][64] bf16
+  static constexpr uint32_t ds = p + 2 * KV_M * Q_N * 2;      // 2 x [128][64] bf16
+  static constexpr uint32_t bar = ds + 2 * KV_M * Q_N * 2;
   static constexpr uint32_t bytes = bar + 256;
 };
 
 struct DkdvBars {
-  uint64_t kvfull, qfull[2], qempty[2], sfull[2], sfree[2], pfull, dsfree, done, lfull[2];
+  uint64_t kvfull, qfull[QST], qempty[QST], sfull[2], sfree[2], pfull, dsfree[2], done;
   uint32_t tmem_base;
 };
 
@@ -68,7 +75,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
   DkdvBars* bars = reinterpret_cast<DkdvBars*>(smem + Lay::bar);
-  float* vec = reinterpret_cast<float*>(smem + Lay::vec);  // [buf][lse|delta][64]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kt = (int)(blockIdx.x / BH);  // key tile 0 walks the most query tiles: first
   const int bh = (int)(blockIdx.x % BH);
@@ -78,15 +84,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kvfull, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < QST; ++s) {
       mbar_init(&bars->qfull[s], 1);
       mbar_init(&bars->qempty[s], 1);
-      mbar_init(&bars->sfull[s], 1);
-      mbar_init(&bars->sfree[s], 128);
-      mbar_init(&bars->lfull[s], Q_N);
     }
-    mbar_init(&bars->pfull, 128);
-    mbar_init(&bars->dsfree, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->sfull[s], 1);
+      mbar_init(&bars->sfree[s], kSoftmax);
+      mbar_init(&bars->dsfree[s], 1);
+    }
+    mbar_init(&bars->pfull, kSoftmax);
     mbar_init(&bars->done, 1);
     fence_mbar_init();
   }
@@ -107,8 +114,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(&tmV, &bars->kvfull, smem + Lay::v + blk * KV_M * 128, 64 * blk, kt * KV_M, bh);
       }
       for (int it = 0; it < n_it; ++it) {
-        const int s = it & 1;
-        if (!mbar_wait(&bars->qempty[s], ((it >> 1) & 1) ^ 1, status, 21)) break;
+        const int s = it % QST;
+        if (!mbar_wait(&bars->qempty[s], ((it / QST) & 1) ^ 1, status, 21)) break;
         mbar_expect_tx(&bars->qfull[s], 2 * Q_N * HD * 2);
         const int row = (i0 + it) * Q_N;
         for (int blk = 0; blk < HD / 64; ++blk) {
@@ -128,27 +135,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sP = smem_u32(smem + Lay::p), sDS = smem_u32(smem + Lay::ds);
       bool ok = mbar_wait(&bars->kvfull, 0, status, 22);
       auto grads = [&](int it) -> bool {
-        const int s = it & 1;
+        const int s = it % QST, pb = it & 1;
         if (!mbar_wait(&bars->pfull, it & 1, status, 23)) return false;
         tc_fence_after();
         const uint32_t qb = sQ + s * Q_N * HD * 2, ob = sO + s * Q_N * HD * 2;
 #pragma unroll
         for (int ks = 0; ks < Q_N / 16; ++ks) {
-          const uint64_t ap = sdesc_sw128(sP + ks * 32, 16, 1024);
-          const uint64_t ad = sdesc_sw128(sDS + ks * 32, 16, 1024);
+          const uint64_t ap = sdesc_sw128(sP + pb * KV_M * Q_N * 2 + ks * 32, 16, 1024);
+          const uint64_t ad = sdesc_sw128(sDS + pb * KV_M * Q_N * 2 + ks * 32, 16, 1024);
           const uint64_t bo = sdesc_sw128(ob + ks * 16 * 128, Q_N * 128, 1024);
           const uint64_t bq = sdesc_sw128(qb + ks * 16 * 128, Q_N * 128, 1024);
           const uint32_t acc = (it > 0 || ks > 0) ? 1u : 0u;
           mma_bf16(tmem + 256, ap, bo, idG, acc);       // dV += P^T dO
           mma_bf16(tmem + 256 + HD, ad, bq, idG, acc);  // dK += dS^T Q
         }
-        mma_commit(&bars->dsfree);
+        mma_commit(&bars->dsfree[pb]);
         mma_commit(&bars->qempty[s]);
         return true;
       };
       for (int it = 0; ok && it < n_it; ++it) {
-        const int s = it & 1, sb = it & 1;
-        if (!mbar_wait(&bars->qfull[s], (it >> 1) & 1, status, 24)) { ok = false; break; }
+        const int s = it % QST, sb = it & 1;
+        if (!mbar_wait(&bars->qfull[s], (it / QST) & 1, status, 24)) { ok = false; break; }
         if (!mbar_wait(&bars->sfree[sb], ((it >> 1) & 1) ^ 1, status, 25)) { ok = false; break; }
         tc_fence_after();
         const uint32_t qb = sQ + s * Q_N * HD * 2, ob = sO + s * Q_N * HD * 2;
@@ -168,62 +175,78 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;                // which 32 of the 64 query columns
     const int r = quarter * 32 + lane;               // key row in the tile
     const int kvrow = kt * KV_M + r;
-    const int st = threadIdx.x - 64;                 // 0..127 among the softmax threads
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
     uint8_t* pP = smem + Lay::p;
     uint8_t* pDS = smem + Lay::ds;
     const float c = scale * kLog2e;
+    const int c0 = half * 32;
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int sb = it & 1;
       const int q0 = (i0 + it) * Q_N;
-      // LSE (log2 units) and D of the tile's 64 query rows, shared through
-      // shared memory.  The buffer used two tiles ago is free: every reader
-      // arrived on pfull for that tile before this thread saw dsfree for it.
-      float* lbuf = vec + sb * 2 * Q_N;
-      if (st < Q_N) {
-        const int qr = q0 + st;
-        lbuf[st] = qr < S ? __ldg(lse + (int64_t)bh * S + qr) * kLog2e : INFINITY;
-        lbuf[Q_N + st] = qr < S ? __ldg(delta + (int64_t)bh * S + qr) : 0.f;
-        mbar_arrive(&bars->lfull[sb]);
+      // LSE (log2 units) and D of this thread's 32 query columns; the
+      // addresses are the same across the warp, so each load is one request
+      // served from L1.  Rows past S get LSE = +inf (P = 0) and D = 0.
+      float lv[32], dv[32];
+      const int qb0 = q0 + c0;
+      const float* lrow = lse + (int64_t)bh * S + qb0;
+      const float* drow = delta + (int64_t)bh * S + qb0;
+      if (qb0 + 32 <= S) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          lv[e] = __ldg(lrow + e) * kLog2e;
+          dv[e] = __ldg(drow + e);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const bool in = qb0 + e < S;
+          lv[e] = in ? __ldg(lrow + e) * kLog2e : INFINITY;
+          dv[e] = in ? __ldg(drow + e) : 0.f;
+        }
       }
-      if (!mbar_wait(&bars->lfull[sb], (it >> 1) & 1, status, 29)) { ok = false; break; }
       if (!mbar_wait(&bars->sfull[sb], (it >> 1) & 1, status, 26)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sr[2][32], pr[2][32];
-      tmem_ld32(tmem + lane_addr + sb * Q_N, sr[0]);
-      tmem_ld32(tmem + lane_addr + sb * Q_N + 32, sr[1]);
-      tmem_ld32(tmem + lane_addr + 128 + sb * Q_N, pr[0]);
-      tmem_ld32(tmem + lane_addr + 128 + sb * Q_N + 32, pr[1]);
+      uint32_t sr[32], pr[32];
+      tmem_ld32(tmem + lane_addr + sb * Q_N + c0, sr);
+      tmem_ld32(tmem + lane_addr + 128 + sb * Q_N + c0, pr);
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&bars->sfree[sb]);
-      const bool diag = q0 < kt * KV_M + KV_M;       // the tile crosses the diagonal
-      uint32_t pk[Q_N / 2], dk[Q_N / 2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h)
+      uint32_t pk[16], dk[16];
+      if (q0 < kt * KV_M + KV_M) {                    // the tile crosses the diagonal
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const int col = h * 32 + e;
-          float p0 = ex2(fmaf(__uint_as_float(sr[h][e]), c, -lbuf[col]));
-          float p1 = ex2(fmaf(__uint_as_float(sr[h][e + 1]), c, -lbuf[col + 1]));
-          if (diag) {
-            p0 = (q0 + col >= kvrow) ? p0 : 0.f;
-            p1 = (q0 + col + 1 >= kvrow) ? p1 : 0.f;
-          }
-          const float d0 = p0 * (__uint_as_float(pr[h][e]) - lbuf[Q_N + col]);
-          const float d1 = p1 * (__uint_as_float(pr[h][e + 1]) - lbuf[Q_N + col + 1]);
-          pk[col >> 1] = pack_bf16x2(p0, p1);
-          dk[col >> 1] = pack_bf16x2(d0, d1);
+          float p0 = ex2(fmaf(__uint_as_float(sr[e]), c, -lv[e]));
+          float p1 = ex2(fmaf(__uint_as_float(sr[e + 1]), c, -lv[e + 1]));
+          p0 = (q0 + c0 + e >= kvrow) ? p0 : 0.f;
+          p1 = (q0 + c0 + e + 1 >= kvrow) ? p1 : 0.f;
+          pk[e >> 1] = pack_bf16x2(p0, p1);
+          dk[e >> 1] = pack_bf16x2(p0 * (__uint_as_float(pr[e]) - dv[e]),
+                                   p1 * (__uint_as_float(pr[e + 1]) - dv[e + 1]));
         }
-      if (it > 0 && !mbar_wait(&bars->dsfree, (it - 1) & 1, status, 27)) { ok = false; break; }
+      } else {
 #pragma unroll
-      for (int cc = 0; cc < 8; ++cc) {
-        const uint32_t off = r * 128 + ((cc ^ (r & 7)) << 4);
-        *reinterpret_cast<uint4*>(pP + off) = make_uint4(pk[cc * 4], pk[cc * 4 + 1], pk[cc * 4 + 2], pk[cc * 4 + 3]);
-        *reinterpret_cast<uint4*>(pDS + off) = make_uint4(dk[cc * 4], dk[cc * 4 + 1], dk[cc * 4 + 2], dk[cc * 4 + 3]);
+        for (int e = 0; e < 32; e += 2) {
+          const float p0 = ex2(fmaf(__uint_as_float(sr[e]), c, -lv[e]));
+          const float p1 = ex2(fmaf(__uint_as_float(sr[e + 1]), c, -lv[e + 1]));
+          pk[e >> 1] = pack_bf16x2(p0, p1);
+          dk[e >> 1] = pack_bf16x2(p0 * (__uint_as_float(pr[e]) - dv[e]),
+                                   p1 * (__uint_as_float(pr[e + 1]) - dv[e + 1]));
+        }
+      }
+      // P / dS buffer it % 2 was last read by the gradient MMAs of tile it - 2
+      const int pb = it & 1;
+      if (it >= 2 && !mbar_wait(&bars->dsfree[pb], ((it >> 1) & 1) ^ 1, status, 27)) { ok = false; break; }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int cc = half * 4 + q;
+        const uint32_t off = pb * KV_M * Q_N * 2 + r * 128 + ((cc ^ (r & 7)) << 4);
+        *reinterpret_cast<uint4*>(pP + off) = make_uint4(pk[q * 4], pk[q * 4 + 1], pk[q * 4 + 2], pk[q * 4 + 3]);
+        *reinterpret_cast<uint4*>(pDS + off) = make_uint4(dk[q * 4], dk[q * 4 + 1], dk[q * 4 + 2], dk[q * 4 + 3]);
       }
       fence_async_smem();
       tc_fence_before();
@@ -231,25 +254,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok && mbar_wait(&bars->done, 0, status, 28)) {
       tc_fence_after();
+      const int which = half;                        // warpgroup 0 writes dV, 1 writes dK
+      uint4* dst = (which ? dkg : dvg) + ((int64_t)bh * S + kvrow) * (HD / 8);
+      const float mul = which ? scale : 1.f;
 #pragma unroll
-      for (int which = 0; which < 2; ++which) {     // 0: dV, 1: dK
-        uint4* dst = (which ? dkg : dvg) + ((int64_t)bh * S + kvrow) * (HD / 8);
-        const float mul = which ? scale : 1.f;
+      for (int cchunk = 0; cchunk < HD / 32; ++cchunk) {
+        uint32_t o[32];
+        tmem_ld32(tmem + lane_addr + 256 + which * HD + cchunk * 32, o);
+        tmem_ld_wait();
+        if (kvrow < S) {
 #pragma unroll
-        for (int cchunk = 0; cchunk < HD / 32; ++cchunk) {
-          uint32_t o[32];
-          tmem_ld32(tmem + lane_addr + 256 + which * HD + cchunk * 32, o);
-          tmem_ld_wait();
-          if (kvrow < S) {
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint4 w;
-              w.x = pack_bf16x2(__uint_as_float(o[v * 8 + 0]) * mul, __uint_as_float(o[v * 8 + 1]) * mul);
-              w.y = pack_bf16x2(__uint_as_float(o[v * 8 + 2]) * mul, __uint_as_float(o[v * 8 + 3]) * mul);
-              w.z = pack_bf16x2(__uint_as_float(o[v * 8 + 4]) * mul, __uint_as_float(o[v * 8 + 5]) * mul);
-              w.w = pack_bf16x2(__uint_as_float(o[v * 8 + 6]) * mul, __uint_as_float(o[v * 8 + 7]) * mul);
-              dst[cchunk * 4 + v] = w;
-            }
+          for (int v = 0; v < 4; ++v) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(o[v * 8 + 0]) * mul, __uint_as_float(o[v * 8 + 1]) * mul);
+            w.y = pack_bf16x2(__uint_as_float(o[v * 8 + 2]) * mul, __uint_as_float(o[v * 8 + 3]) * mul);
+            w.z = pack_bf16x2(__uint_as_float(o[v * 8 + 4]) * mul, __uint_as_float(o[v * 8 + 5]) * mul);
+            w.w = pack_bf16x2(__uint_as_float(o[v * 8 + 6]) * mul, __uint_as_float(o[v * 8 + 7]) * mul);
+            dst[cchunk * 4 + v] = w;
           }
         }
       }
@@ -268,19 +289,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 constexpr int Q_M = 128;   // stationary query rows
 constexpr int KV_N = 64;   // walked key rows per tile
 
+constexpr int KST = 4;     // stages of the walked K / V ring
+
 template <int HD>
 struct DqLayout {
   static constexpr uint32_t q = 0;
   static constexpr uint32_t dO = q + Q_M * HD * 2;
-  static constexpr uint32_t k = dO + Q_M * HD * 2;          // 2 stages
-  static constexpr uint32_t v = k + 2 * KV_N * HD * 2;       // 2 stages
-  static constexpr uint32_t ds = v + 2 * KV_N * HD * 2;      // [128][64] bf16
-  static constexpr uint32_t bar = ds + Q_M * KV_N * 2;
+  static constexpr uint32_t k = dO + Q_M * HD * 2;          // KST stages
+  static constexpr uint32_t v = k + KST * KV_N * HD * 2;     // KST stages
+  static constexpr uint32_t ds = v + KST * KV_N * HD * 2;    // 2 x [128][64] bf16
+  static constexpr uint32_t bar = ds + 2 * Q_M * KV_N * 2;
   static constexpr uint32_t bytes = bar + 256;
 };
 
 struct DqBars {
-  uint64_t qfull, kvfull[2], kvempty[2], sfull[2], sfree[2], pfull, dsfree, done;
+  uint64_t qfull, kvfull[KST], kvempty[KST], sfull[2], sfree[2], pfull, dsfree[2], done;
   uint32_t tmem_base;
 };
 
@@ -304,14 +327,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->qfull, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < KST; ++s) {
       mbar_init(&bars->kvfull[s], 1);
       mbar_init(&bars->kvempty[s], 1);
-      mbar_init(&bars->sfull[s], 1);
-      mbar_init(&bars->sfree[s], 128);
     }
-    mbar_init(&bars->pfull, 128);
-    mbar_init(&bars->dsfree, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->sfull[s], 1);
+      mbar_init(&bars->sfree[s], kSoftmax);
+      mbar_init(&bars->dsfree[s], 1);
+    }
+    mbar_init(&bars->pfull, kSoftmax);
     mbar_init(&bars->done, 1);
     fence_mbar_init();
   }
@@ -332,8 +357,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(&tmO, &bars->qfull, smem + Lay::dO + blk * Q_M * 128, 64 * blk, qt * Q_M, bh);
       }
       for (int j = 0; j < n_kv; ++j) {
-        const int s = j & 1;
-        if (!mbar_wait(&bars->kvempty[s], ((j >> 1) & 1) ^ 1, status, 31)) break;
+        const int s = j % KST;
+        if (!mbar_wait(&bars->kvempty[s], ((j / KST) & 1) ^ 1, status, 31)) break;
         mbar_expect_tx(&bars->kvfull[s], 2 * KV_N * HD * 2);
         for (int blk = 0; blk < HD / 64; ++blk) {
           tma_load_3d(&tmK, &bars->kvfull[s], smem + Lay::k + s * KV_N * HD * 2 + blk * KV_N * 128,
@@ -352,22 +377,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sDS = smem_u32(smem + Lay::ds);
       bool ok = mbar_wait(&bars->qfull, 0, status, 32);
       auto grad = [&](int j) -> bool {
-        const int s = j & 1;
+        const int s = j % KST, pb = j & 1;
         if (!mbar_wait(&bars->pfull, j & 1, status, 33)) return false;
         tc_fence_after();
         const uint32_t kb = sK + s * KV_N * HD * 2;
 #pragma unroll
         for (int ks = 0; ks < KV_N / 16; ++ks)
-          mma_bf16(tmem + 256, sdesc_sw128(sDS + ks * 32, 16, 1024),
+          mma_bf16(tmem + 256, sdesc_sw128(sDS + pb * Q_M * KV_N * 2 + ks * 32, 16, 1024),
                    sdesc_sw128(kb + ks * 16 * 128, KV_N * 128, 1024), idG,
                    (j > 0 || ks > 0) ? 1u : 0u);
-        mma_commit(&bars->dsfree);
+        mma_commit(&bars->dsfree[pb]);
         mma_commit(&bars->kvempty[s]);
         return true;
       };
       for (int j = 0; ok && j < n_kv; ++j) {
-        const int s = j & 1, sb = j & 1;
-        if (!mbar_wait(&bars->kvfull[s], (j >> 1) & 1, status, 34)) { ok = false; break; }
+        const int s = j % KST, sb = j & 1;
+        if (!mbar_wait(&bars->kvfull[s], (j / KST) & 1, status, 34)) { ok = false; break; }
         if (!mbar_wait(&bars->sfree[sb], ((j >> 1) & 1) ^ 1, status, 35)) { ok = false; break; }
         tc_fence_after();
         const uint32_t kb = sK + s * KV_N * HD * 2, vb = sV + s * KV_N * HD * 2;
@@ -387,11 +412,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;                // which 32 of the 64 key columns
     const int r = quarter * 32 + lane;
     const int qrow = qt * Q_M + r;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
     uint8_t* pDS = smem + Lay::ds;
     const float c = scale * kLog2e;
+    const int c0 = half * 32;
     const float lrow = qrow < S ? __ldg(lse + (int64_t)bh * S + qrow) * kLog2e : INFINITY;
     const float drow = qrow < S ? __ldg(delta + (int64_t)bh * S + qrow) : 0.f;
     bool ok = true;
@@ -400,35 +427,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int k0 = j * KV_N;
       if (!mbar_wait(&bars->sfull[sb], (j >> 1) & 1, status, 36)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sr[2][32], pr[2][32];
-      tmem_ld32(tmem + lane_addr + sb * KV_N, sr[0]);
-      tmem_ld32(tmem + lane_addr + sb * KV_N + 32, sr[1]);
-      tmem_ld32(tmem + lane_addr + 128 + sb * KV_N, pr[0]);
-      tmem_ld32(tmem + lane_addr + 128 + sb * KV_N + 32, pr[1]);
+      uint32_t sr[32], pr[32];
+      tmem_ld32(tmem + lane_addr + sb * KV_N + c0, sr);
+      tmem_ld32(tmem + lane_addr + 128 + sb * KV_N + c0, pr);
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&bars->sfree[sb]);
-      const bool diag = k0 + KV_N > qt * Q_M;
-      uint32_t dk[KV_N / 2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h)
+      uint32_t dk[16];
+      if (k0 + KV_N > qt * Q_M) {                     // the tile crosses the diagonal
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const int col = h * 32 + e;
-          float p0 = ex2(fmaf(__uint_as_float(sr[h][e]), c, -lrow));
-          float p1 = ex2(fmaf(__uint_as_float(sr[h][e + 1]), c, -lrow));
-          if (diag) {
-            p0 = (k0 + col <= qrow) ? p0 : 0.f;
-            p1 = (k0 + col + 1 <= qrow) ? p1 : 0.f;
-          }
-          dk[col >> 1] = pack_bf16x2(p0 * (__uint_as_float(pr[h][e]) - drow),
-                                     p1 * (__uint_as_float(pr[h][e + 1]) - drow));
+          float p0 = ex2(fmaf(__uint_as_float(sr[e]), c, -lrow));
+          float p1 = ex2(fmaf(__uint_as_float(sr[e + 1]), c, -lrow));
+          p0 = (k0 + c0 + e <= qrow) ? p0 : 0.f;
+          p1 = (k0 + c0 + e + 1 <= qrow) ? p1 : 0.f;
+          dk[e >> 1] = pack_bf16x2(p0 * (__uint_as_float(pr[e]) - drow),
+                                   p1 * (__uint_as_float(pr[e + 1]) - drow));
         }
-      if (j > 0 && !mbar_wait(&bars->dsfree, (j - 1) & 1, status, 37)) { ok = false; break; }
+      } else {
 #pragma unroll
-      for (int cc = 0; cc < 8; ++cc)
-        *reinterpret_cast<uint4*>(pDS + r * 128 + ((cc ^ (r & 7)) << 4)) =
-            make_uint4(dk[cc * 4], dk[cc * 4 + 1], dk[cc * 4 + 2], dk[cc * 4 + 3]);
+        for (int e = 0; e < 32; e += 2) {
+          const float p0 = ex2(fmaf(__uint_as_float(sr[e]), c, -lrow));
+          const float p1 = ex2(fmaf(__uint_as_float(sr[e + 1]), c, -lrow));
+          dk[e >> 1] = pack_bf16x2(p0 * (__uint_as_float(pr[e]) - drow),
+                                   p1 * (__uint_as_float(pr[e + 1]) - drow));
+        }
+      }
+      // dS buffer j % 2 was last read by the dQ MMAs of tile j - 2
+      const int pb = j & 1;
+      if (j >= 2 && !mbar_wait(&bars->dsfree[pb], ((j >> 1) & 1) ^ 1, status, 37)) { ok = false; break; }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int cc = half * 4 + q;
+        *reinterpret_cast<uint4*>(pDS + pb * Q_M * KV_N * 2 + r * 128 + ((cc ^ (r & 7)) << 4)) =
+            make_uint4(dk[q * 4], dk[q * 4 + 1], dk[q * 4 + 2], dk[q * 4 + 3]);
+      }
       fence_async_smem();
       tc_fence_before();
       mbar_arrive(&bars->pfull);
@@ -437,7 +470,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       uint4* dst = dqg + ((int64_t)bh * S + qrow) * (HD / 8);
 #pragma unroll
-      for (int cchunk = 0; cchunk < HD / 32; ++cchunk) {
+      for (int q = 0; q < HD / 64; ++q) {            // each warpgroup: half of the d columns
+        const int cchunk = half * (HD / 64) + q;
         uint32_t o[32];
         tmem_ld32(tmem + lane_addr + 256 + cchunk * 32, o);
         tmem_ld_wait();

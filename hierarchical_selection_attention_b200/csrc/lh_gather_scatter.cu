@@ -43,7 +43,9 @@ __device__ __forceinline__ const uint4* level_row(const LhDims& D, const uint4* 
   return xl + (((int64_t)D.B * D.pool_row[l] + (int64_t)b * D.lvl_size[l] + i) * D.H + h) * V;
 }
 
-// (iii) gather: thread = (b, h, slot m, vector cv).
+// (iii) gather: thread = (b, h, slot m, vector cv).  I is the index type:
+// 32-bit whenever the item count fits, which keeps the div/mod cheap.
+template <typename I>
 __global__ void __launch_bounds__(kThreads) k_gather(LhDims D, const uint4* __restrict__ q,
                                                      const uint4* __restrict__ k,
                                                      const uint4* __restrict__ v,
@@ -54,12 +56,12 @@ __global__ void __launch_bounds__(kThreads) k_gather(LhDims D, const uint4* __re
                                                      uint4* __restrict__ qg, uint4* __restrict__ kg,
                                                      uint4* __restrict__ vg) {
   const int V = D.d >> 3;
-  const int64_t item = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t total = (int64_t)D.B * D.H * D.S * V;
+  const I item = (I)blockIdx.x * blockDim.x + threadIdx.x;
+  const I total = (I)D.B * D.H * D.S * V;
   if (item >= total) return;
-  const int cv = (int)(item % V);
-  const int64_t row = item / V;  // (bh, m)
-  const int64_t bh = row / D.S;
+  const int cv = (int)(item & (V - 1));
+  const I row = item / V;  // (bh, m)
+  const I bh = row / (I)D.S;
   const int b = (int)(bh / D.H), h = (int)(bh % D.H);
   const int64_t f = __ldg(sel_idx + row);
   if (f < 0 || f >= D.P) {
@@ -68,7 +70,7 @@ __global__ void __launch_bounds__(kThreads) k_gather(LhDims D, const uint4* __re
   }
   const int l = lh_level_of(D, f);
   const int64_t i = f - D.lvl_off[l];
-  const int64_t o = row * V + cv;
+  const int64_t o = (int64_t)row * V + cv;
   qg[o] = __ldg(level_row(D, q, q_lv, l, b, i, h, V) + cv);
   kg[o] = __ldg(level_row(D, k, k_lv, l, b, i, h, V) + cv);
   vg[o] = __ldg(level_row(D, v, v_lv, l, b, i, h, V) + cv);
@@ -78,20 +80,20 @@ __global__ void __launch_bounds__(kThreads) k_gather(LhDims D, const uint4* __re
 // level l that reaches t is i = floor((t+1)/p^l) - 1.  All slot lookups are
 // issued before any row load, and all row loads before the sum, so a thread
 // waits for two memory round trips rather than two per level.
-template <int L>
+template <int L, typename I>
 __global__ void __launch_bounds__(kThreads) k_scatter(LhDims D, const uint4* __restrict__ og,
                                                       const int32_t* __restrict__ slot_map,
                                                       uint4* __restrict__ o) {
   const int V = D.d >> 3;
-  const int64_t item = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t total = (int64_t)D.B * D.N * D.H * V;
+  const I item = (I)blockIdx.x * blockDim.x + threadIdx.x;
+  const I total = (I)D.B * D.N * D.H * V;
   if (item >= total) return;
-  const int cv = (int)(item % V);
-  const int64_t r = item / V;  // (b, t, h)
-  const int h = (int)(r % D.H);
-  const int64_t bt = r / D.H;
-  const int64_t t = bt % D.N;
-  const int b = (int)(bt / D.N);
+  const int cv = (int)(item & (V - 1));
+  const I r = item / V;  // (b, t, h)
+  const int h = (int)(r % (I)D.H);
+  const I bt = r / (I)D.H;
+  const int64_t t = (int64_t)(bt % (I)D.N);
+  const int b = (int)(bt / (I)D.N);
   const int64_t bh = (int64_t)b * D.H + h;
   const int32_t* sm = slot_map + bh * D.P;
   const uint4* src = og + bh * D.S * V + cv;
@@ -159,6 +161,7 @@ __global__ void __launch_bounds__(kThreads) k_scatter_fix2bf16(int64_t n,
 
 // Adjoint of the scatter, fused with D = rowsum(dog * og): thread = (b, h,
 // slot m, vector cv); it sums dO over the shifted range of the slot's entry.
+template <typename I>
 __global__ void __launch_bounds__(kThreads) k_scatter_bwd(LhDims D, const uint4* __restrict__ dout,
                                                           const uint4* __restrict__ og,
                                                           const uint4* __restrict__ og_lo,
@@ -166,13 +169,13 @@ __global__ void __launch_bounds__(kThreads) k_scatter_bwd(LhDims D, const uint4*
                                                           uint4* __restrict__ dog,
                                                           float* __restrict__ delta) {
   const int V = D.d >> 3;
-  const int64_t item = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t total = (int64_t)D.B * D.H * D.S * V;
+  const I item = (I)blockIdx.x * blockDim.x + threadIdx.x;
+  const I total = (I)D.B * D.H * D.S * V;
   const unsigned live = __ballot_sync(0xffffffffu, item < total);
   if (item >= total) return;
-  const int cv = (int)(item % V);
-  const int64_t row = item / V;
-  const int64_t bh = row / D.S;
+  const int cv = (int)(item & (V - 1));
+  const I row = item / V;
+  const I bh = row / (I)D.S;
   const int b = (int)(bh / D.H), h = (int)(bh % D.H);
   const int64_t f = __ldg(sel_idx + row);
   const int l = lh_level_of(D, f);
@@ -229,7 +232,7 @@ __global__ void __launch_bounds__(kThreads) k_attn_delta(int64_t rows, int V,
 // Adjoint of gather + mean pooling: thread = (b, t, h, vector cv); the level-l
 // entry whose (unshifted) window holds t is i = floor(t / p^l).  Slot lookups
 // first, then every row load, then the sums (two memory round trips).
-template <int L>
+template <int L, typename I>
 __global__ void __launch_bounds__(kThreads) k_gather_bwd(LhDims D, const uint4* __restrict__ dqg,
                                                          const uint4* __restrict__ dkg,
                                                          const uint4* __restrict__ dvg,
@@ -237,15 +240,15 @@ __global__ void __launch_bounds__(kThreads) k_gather_bwd(LhDims D, const uint4* 
                                                          uint4* __restrict__ dq, uint4* __restrict__ dk,
                                                          uint4* __restrict__ dv) {
   const int V = D.d >> 3;
-  const int64_t item = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t total = (int64_t)D.B * D.N * D.H * V;
+  const I item = (I)blockIdx.x * blockDim.x + threadIdx.x;
+  const I total = (I)D.B * D.N * D.H * V;
   if (item >= total) return;
-  const int cv = (int)(item % V);
-  const int64_t r = item / V;
-  const int h = (int)(r % D.H);
-  const int64_t bt = r / D.H;
-  const int64_t t = bt % D.N;
-  const int b = (int)(bt / D.N);
+  const int cv = (int)(item & (V - 1));
+  const I r = item / V;
+  const int h = (int)(r % (I)D.H);
+  const I bt = r / (I)D.H;
+  const int64_t t = (int64_t)(bt % (I)D.N);
+  const int b = (int)(bt / (I)D.N);
   const int64_t bh = (int64_t)b * D.H + h;
   const int32_t* sm = slot_map + bh * D.P;
   int slot[L];
@@ -279,6 +282,39 @@ __global__ void __launch_bounds__(kThreads) k_gather_bwd(LhDims D, const uint4* 
 
 inline unsigned nblocks(int64_t n) { return (unsigned)((n + kThreads - 1) / kThreads); }
 
+constexpr int64_t kIdx32 = (int64_t)1 << 31;  // item counts below this use 32-bit indices
+
+template <typename I>
+cudaError_t scatter_L(const LhDims& D, unsigned g, const uint4* x, const int32_t* sm, uint4* o,
+                      cudaStream_t st) {
+  switch (D.L) {
+    case 1: k_scatter<1, I><<<g, kThreads, 0, st>>>(D, x, sm, o); break;
+    case 2: k_scatter<2, I><<<g, kThreads, 0, st>>>(D, x, sm, o); break;
+    case 3: k_scatter<3, I><<<g, kThreads, 0, st>>>(D, x, sm, o); break;
+    case 4: k_scatter<4, I><<<g, kThreads, 0, st>>>(D, x, sm, o); break;
+    case 5: k_scatter<5, I><<<g, kThreads, 0, st>>>(D, x, sm, o); break;
+    case 6: k_scatter<6, I><<<g, kThreads, 0, st>>>(D, x, sm, o); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+template <typename I>
+cudaError_t gather_bwd_L(const LhDims& D, unsigned g, const uint4* a, const uint4* b,
+                         const uint4* c, const int32_t* sm, uint4* x, uint4* y, uint4* z,
+                         cudaStream_t st) {
+  switch (D.L) {
+    case 1: k_gather_bwd<1, I><<<g, kThreads, 0, st>>>(D, a, b, c, sm, x, y, z); break;
+    case 2: k_gather_bwd<2, I><<<g, kThreads, 0, st>>>(D, a, b, c, sm, x, y, z); break;
+    case 3: k_gather_bwd<3, I><<<g, kThreads, 0, st>>>(D, a, b, c, sm, x, y, z); break;
+    case 4: k_gather_bwd<4, I><<<g, kThreads, 0, st>>>(D, a, b, c, sm, x, y, z); break;
+    case 5: k_gather_bwd<5, I><<<g, kThreads, 0, st>>>(D, a, b, c, sm, x, y, z); break;
+    case 6: k_gather_bwd<6, I><<<g, kThreads, 0, st>>>(D, a, b, c, sm, x, y, z); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t lh_launch_gather(const LhDims& D, const lh_bf16* q, const lh_bf16* k,
@@ -286,9 +322,14 @@ cudaError_t lh_launch_gather(const LhDims& D, const lh_bf16* q, const lh_bf16* k
                              const lh_bf16* v_lv, const int32_t* sel_idx, lh_bf16* qg,
                              lh_bf16* kg, lh_bf16* vg, cudaStream_t st) {
   const int64_t n = (int64_t)D.B * D.H * D.S * (D.d >> 3);
-  k_gather<<<nblocks(n), kThreads, 0, st>>>(
-      D, (const uint4*)q, (const uint4*)k, (const uint4*)v, (const uint4*)q_lv,
-      (const uint4*)k_lv, (const uint4*)v_lv, sel_idx, (uint4*)qg, (uint4*)kg, (uint4*)vg);
+  if (n < kIdx32)
+    k_gather<uint32_t><<<nblocks(n), kThreads, 0, st>>>(
+        D, (const uint4*)q, (const uint4*)k, (const uint4*)v, (const uint4*)q_lv,
+        (const uint4*)k_lv, (const uint4*)v_lv, sel_idx, (uint4*)qg, (uint4*)kg, (uint4*)vg);
+  else
+    k_gather<uint64_t><<<nblocks(n), kThreads, 0, st>>>(
+        D, (const uint4*)q, (const uint4*)k, (const uint4*)v, (const uint4*)q_lv,
+        (const uint4*)k_lv, (const uint4*)v_lv, sel_idx, (uint4*)qg, (uint4*)kg, (uint4*)vg);
   return cudaGetLastError();
 }
 
@@ -297,16 +338,8 @@ cudaError_t lh_launch_scatter(const LhDims& D, const lh_bf16* og, const int32_t*
   const int64_t n = (int64_t)D.B * D.N * D.H * (D.d >> 3);
   const unsigned g = nblocks(n);
   const uint4* x = (const uint4*)og;
-  switch (D.L) {
-    case 1: k_scatter<1><<<g, kThreads, 0, st>>>(D, x, slot_map, (uint4*)o); break;
-    case 2: k_scatter<2><<<g, kThreads, 0, st>>>(D, x, slot_map, (uint4*)o); break;
-    case 3: k_scatter<3><<<g, kThreads, 0, st>>>(D, x, slot_map, (uint4*)o); break;
-    case 4: k_scatter<4><<<g, kThreads, 0, st>>>(D, x, slot_map, (uint4*)o); break;
-    case 5: k_scatter<5><<<g, kThreads, 0, st>>>(D, x, slot_map, (uint4*)o); break;
-    case 6: k_scatter<6><<<g, kThreads, 0, st>>>(D, x, slot_map, (uint4*)o); break;
-    default: return cudaErrorInvalidValue;
-  }
-  return cudaGetLastError();
+  if (n < kIdx32) return scatter_L<uint32_t>(D, g, x, slot_map, (uint4*)o, st);
+  return scatter_L<uint64_t>(D, g, x, slot_map, (uint4*)o, st);
 }
 
 size_t lh_scatter_atomic_ws_bytes(const LhDims& D) {
@@ -332,8 +365,12 @@ cudaError_t lh_launch_scatter_bwd(const LhDims& D, const lh_bf16* dout, const lh
                                   const lh_bf16* og_lo, const int32_t* sel_idx, lh_bf16* dog,
                                   float* delta, cudaStream_t st) {
   const int64_t n = (int64_t)D.B * D.H * D.S * (D.d >> 3);
-  k_scatter_bwd<<<nblocks(n), kThreads, 0, st>>>(D, (const uint4*)dout, (const uint4*)og,
-                                                 (const uint4*)og_lo, sel_idx, (uint4*)dog, delta);
+  if (n < kIdx32)
+    k_scatter_bwd<uint32_t><<<nblocks(n), kThreads, 0, st>>>(
+        D, (const uint4*)dout, (const uint4*)og, (const uint4*)og_lo, sel_idx, (uint4*)dog, delta);
+  else
+    k_scatter_bwd<uint64_t><<<nblocks(n), kThreads, 0, st>>>(
+        D, (const uint4*)dout, (const uint4*)og, (const uint4*)og_lo, sel_idx, (uint4*)dog, delta);
   return cudaGetLastError();
 }
 
@@ -354,14 +391,6 @@ cudaError_t lh_launch_gather_bwd(const LhDims& D, const lh_bf16* dqg, const lh_b
   const unsigned g = nblocks(n);
   const uint4 *a = (const uint4*)dqg, *b = (const uint4*)dkg, *c = (const uint4*)dvg;
   uint4 *x = (uint4*)dq, *y = (uint4*)dk, *z = (uint4*)dv;
-  switch (D.L) {
-    case 1: k_gather_bwd<1><<<g, kThreads, 0, st>>>(D, a, b, c, slot_map, x, y, z); break;
-    case 2: k_gather_bwd<2><<<g, kThreads, 0, st>>>(D, a, b, c, slot_map, x, y, z); break;
-    case 3: k_gather_bwd<3><<<g, kThreads, 0, st>>>(D, a, b, c, slot_map, x, y, z); break;
-    case 4: k_gather_bwd<4><<<g, kThreads, 0, st>>>(D, a, b, c, slot_map, x, y, z); break;
-    case 5: k_gather_bwd<5><<<g, kThreads, 0, st>>>(D, a, b, c, slot_map, x, y, z); break;
-    case 6: k_gather_bwd<6><<<g, kThreads, 0, st>>>(D, a, b, c, slot_map, x, y, z); break;
-    default: return cudaErrorInvalidValue;
-  }
-  return cudaGetLastError();
+  if (n < kIdx32) return gather_bwd_L<uint32_t>(D, g, a, b, c, slot_map, x, y, z, st);
+  return gather_bwd_L<uint64_t>(D, g, a, b, c, slot_map, x, y, z, st);
 }
