@@ -58,7 +58,10 @@ struct DkdvLayout {
 };
 
 struct DkdvBars {
-  uint64_t kvfull, qfull[QST], qempty[QST], sfull[2], sfree[2], pfull, dsfree[2], done;
+  // pfull is indexed by tile parity like the P/dS buffers: the softmax of
+  // tile i + 1 may finish before the issuer has seen tile i's phase, and a
+  // single barrier would then complete twice and hide phase i from it.
+  uint64_t kvfull, qfull[QST], qempty[QST], sfull[2], sfree[2], pfull[2], dsfree[2], done;
   uint32_t tmem_base;
 };
 
@@ -92,8 +95,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->sfull[s], 1);
       mbar_init(&bars->sfree[s], kSoftmax);
       mbar_init(&bars->dsfree[s], 1);
+      mbar_init(&bars->pfull[s], kSoftmax);
     }
-    mbar_init(&bars->pfull, kSoftmax);
     mbar_init(&bars->done, 1);
     fence_mbar_init();
   }
@@ -136,7 +139,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = mbar_wait(&bars->kvfull, 0, status, 22);
       auto grads = [&](int it) -> bool {
         const int s = it % QST, pb = it & 1;
-        if (!mbar_wait(&bars->pfull, it & 1, status, 23)) return false;
+        if (!mbar_wait(&bars->pfull[pb], (it >> 1) & 1, status, 23)) return false;
         tc_fence_after();
         const uint32_t qb = sQ + s * Q_N * HD * 2, ob = sO + s * Q_N * HD * 2;
 #pragma unroll
@@ -250,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_async_smem();
       tc_fence_before();
-      mbar_arrive(&bars->pfull);
+      mbar_arrive(&bars->pfull[pb]);
     }
     if (ok && mbar_wait(&bars->done, 0, status, 28)) {
       tc_fence_after();
@@ -297,17 +300,18 @@ struct DqLayout {
   static constexpr uint32_t dO = q + Q_M * HD * 2;
   static constexpr uint32_t k = dO + Q_M * HD * 2;          // KST stages
   static constexpr uint32_t v = k + KST * KV_N * HD * 2;     // KST stages
-  static constexpr uint32_t ds = v + KST * KV_N * HD * 2;    // 2 x [128][64] bf16
-  static constexpr uint32_t bar = ds + 2 * Q_M * KV_N * 2;
+  static constexpr uint32_t bar = v + KST * KV_N * HD * 2;
   static constexpr uint32_t bytes = bar + 256;
 };
 
 struct DqBars {
-  uint64_t qfull, kvfull[KST], kvempty[KST], sfull[2], sfree[2], pfull, dsfree[2], done;
+  // pfull per tile parity, for the reason given at DkdvBars
+  uint64_t qfull, kvfull[KST], kvempty[KST], sfull[2], sfree[2], pfull[2], dsfree[2], done;
   uint32_t tmem_base;
 };
 
-// Columns: S buffers 0/64, dP buffers 128/192, dQ 256.
+// Columns: S buffers 0/64, dP buffers 128/192, dQ 256, dS (bf16 pairs)
+// buffers 384/416.
 template <int HD>
 __global__ void __launch_bounds__(kThreads, 1)
     k_attn_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -335,8 +339,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->sfull[s], 1);
       mbar_init(&bars->sfree[s], kSoftmax);
       mbar_init(&bars->dsfree[s], 1);
+      mbar_init(&bars->pfull[s], kSoftmax);
     }
-    mbar_init(&bars->pfull, kSoftmax);
     mbar_init(&bars->done, 1);
     fence_mbar_init();
   }
@@ -374,18 +378,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idG = idesc_bf16(Q_M, HD, 0, 1);     // dQ (B = K, MN-major)
       const uint32_t sQ = smem_u32(smem + Lay::q), sO = smem_u32(smem + Lay::dO);
       const uint32_t sK = smem_u32(smem + Lay::k), sV = smem_u32(smem + Lay::v);
-      const uint32_t sDS = smem_u32(smem + Lay::ds);
       bool ok = mbar_wait(&bars->qfull, 0, status, 32);
       auto grad = [&](int j) -> bool {
         const int s = j % KST, pb = j & 1;
-        if (!mbar_wait(&bars->pfull, j & 1, status, 33)) return false;
+        if (!mbar_wait(&bars->pfull[pb], (j >> 1) & 1, status, 33)) return false;
         tc_fence_after();
         const uint32_t kb = sK + s * KV_N * HD * 2;
 #pragma unroll
         for (int ks = 0; ks < KV_N / 16; ++ks)
-          mma_bf16(tmem + 256, sdesc_sw128(sDS + pb * Q_M * KV_N * 2 + ks * 32, 16, 1024),
-                   sdesc_sw128(kb + ks * 16 * 128, KV_N * 128, 1024), idG,
-                   (j > 0 || ks > 0) ? 1u : 0u);
+          mma_bf16_ts(tmem + 256, tmem + 384 + pb * 32 + ks * 8,
+                      sdesc_sw128(kb + ks * 16 * 128, KV_N * 128, 1024), idG,
+                      (j > 0 || ks > 0) ? 1u : 0u);
         mma_commit(&bars->dsfree[pb]);
         mma_commit(&bars->kvempty[s]);
         return true;
@@ -416,7 +419,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = quarter * 32 + lane;
     const int qrow = qt * Q_M + r;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-    uint8_t* pDS = smem + Lay::ds;
     const float c = scale * kLog2e;
     const int c0 = half * 32;
     const float lrow = qrow < S ? __ldg(lse + (int64_t)bh * S + qrow) * kLog2e : INFINITY;
@@ -453,18 +455,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                                    p1 * (__uint_as_float(pr[e + 1]) - drow));
         }
       }
-      // dS buffer j % 2 was last read by the dQ MMAs of tile j - 2
+      // dS buffer j % 2 (TMEM) was last read by the dQ MMAs of tile j - 2
       const int pb = j & 1;
       if (j >= 2 && !mbar_wait(&bars->dsfree[pb], ((j >> 1) & 1) ^ 1, status, 37)) { ok = false; break; }
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int cc = half * 4 + q;
-        *reinterpret_cast<uint4*>(pDS + pb * Q_M * KV_N * 2 + r * 128 + ((cc ^ (r & 7)) << 4)) =
-            make_uint4(dk[q * 4], dk[q * 4 + 1], dk[q * 4 + 2], dk[q * 4 + 3]);
-      }
-      fence_async_smem();
+      tmem_st16(tmem + lane_addr + 384 + pb * 32 + half * 16, dk);
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bars->pfull);
+      mbar_arrive(&bars->pfull[pb]);
     }
     if (ok && mbar_wait(&bars->done, 0, status, 38)) {
       tc_fence_after();
