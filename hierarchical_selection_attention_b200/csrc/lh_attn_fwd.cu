@@ -195,24 +195,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int j = 0; j < n_x; ++j) {
       if (!mbar_wait(&bars->sfull[x], j & 1, status, 8)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sr[BN / 32][32];
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) tmem_ld32(tS + c * 32, sr[c]);
-      tmem_ld_wait();
+      // Two passes over the score row in TMEM, two 32-column chunks at a
+      // time: the max first, then exp2 / sum / pack.  Holding the whole row
+      // in registers would spill at this block size.
       const bool diag = (j == qt);
-      float mx = -INFINITY;
-      if (diag) {
+      float mxv[8];
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c)
+      for (int u = 0; u < 8; ++u) mxv[u] = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < BN / 32; c += 2) {
+        uint32_t a[32], b[32];
+        tmem_ld32(tS + c * 32, a);
+        tmem_ld32(tS + c * 32 + 32, b);
+        tmem_ld_wait();
+        if (diag) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            if (c * 32 + e <= r) mxv[e & 7] = fmaxf(mxv[e & 7], __uint_as_float(a[e]));
+            if (c * 32 + 32 + e <= r) mxv[e & 7] = fmaxf(mxv[e & 7], __uint_as_float(b[e]));
+          }
+        } else {
 #pragma unroll
           for (int e = 0; e < 32; ++e)
-            if (c * 32 + e <= r) mx = fmaxf(mx, __uint_as_float(sr[c][e]));
-      } else {
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c)
-#pragma unroll
-          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[c][e]));
+            mxv[e & 7] = fmaxf(mxv[e & 7], fmaxf(__uint_as_float(a[e]), __uint_as_float(b[e])));
+        }
       }
+      const float mx = fmaxf(fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3])),
+                             fmaxf(fmaxf(mxv[4], mxv[5]), fmaxf(mxv[6], mxv[7])));
       // Exact running max: the row's largest term so far gets p = 1, which
       // bf16 holds exactly.  (A stale max, as lazy rescaling keeps, would
       // round that dominant term by up to 2^-9, and the error would reach
@@ -221,23 +230,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool grow = m_new > m_used;
       const float alpha = grow ? ex2(m_used - m_new) : 1.f;
       m_used = m_new;
-      float rs = 0.f;
+      float rsv[8];
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t pk[16];
+      for (int u = 0; u < 8; ++u) rsv[u] = 0.f;
+#pragma unroll
+      for (int c = 0; c < BN / 32; c += 2) {
+        uint32_t a[32], b[32];
+        tmem_ld32(tS + c * 32, a);
+        tmem_ld32(tS + c * 32 + 32, b);
+        tmem_ld_wait();
+        uint32_t pa[16], pb[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          float p0 = ex2(fmaf(__uint_as_float(sr[c][e]), scale_log2, -m_used));
-          float p1 = ex2(fmaf(__uint_as_float(sr[c][e + 1]), scale_log2, -m_used));
+          float p0 = ex2(fmaf(__uint_as_float(a[e]), scale_log2, -m_used));
+          float p1 = ex2(fmaf(__uint_as_float(a[e + 1]), scale_log2, -m_used));
+          float q0 = ex2(fmaf(__uint_as_float(b[e]), scale_log2, -m_used));
+          float q1 = ex2(fmaf(__uint_as_float(b[e + 1]), scale_log2, -m_used));
           if (diag) {
             p0 = (c * 32 + e <= r) ? p0 : 0.f;
             p1 = (c * 32 + e + 1 <= r) ? p1 : 0.f;
+            q0 = (c * 32 + 32 + e <= r) ? q0 : 0.f;
+            q1 = (c * 32 + 32 + e + 1 <= r) ? q1 : 0.f;
           }
-          rs += p0 + p1;
-          pk[e >> 1] = pack_bf16x2(p0, p1);
+          rsv[(e >> 1) & 7] += (p0 + p1) + (q0 + q1);
+          pa[e >> 1] = pack_bf16x2(p0, p1);
+          pb[e >> 1] = pack_bf16x2(q0, q1);
         }
-        tmem_st16(tS + c * 16, pk);  // P over the score columns already read
+        // P over columns of this row already read (pair c covers 64 score
+        // columns from c * 32 and packs into 32 columns from c * 16)
+        tmem_st16(tS + c * 16, pa);
+        tmem_st16(tS + c * 16 + 16, pb);
       }
+      const float rs = ((rsv[0] + rsv[1]) + (rsv[2] + rsv[3])) + ((rsv[4] + rsv[5]) + (rsv[6] + rsv[7]));
       lsum = lsum * alpha + rs;
       // O_X holds P V of the earlier tiles (P_X V of tile j-1 finished before
       // S_X of tile j was issued); bring it to the new max.

@@ -49,16 +49,19 @@ def head(x: torch.Tensor, b: int, h: int) -> np.ndarray:
     return np.ascontiguousarray(x[b, :, h, :].to(torch.float64).cpu().numpy())
 
 
-def attn_bwd_envelopes(qg, kg, vg, dog, scale, chunk=256):
+def attn_bwd_envelopes(qg, kg, vg, dog, scale, chunk=256, rows=None):
     """Magnitude envelopes of the attention gradients: the sums that make
     each gradient with every term replaced by its magnitude.  dS = P dP - P D
     is formed from two products, so its envelope is P (|dP| + |D|):
-    scale P(|dP|+|D|) |K|, scale (P(|dP|+|D|))^T |Q| and P^T |dO| (fp64)."""
+    scale P(|dP|+|D|) |K|, scale (P(|dP|+|D|))^T |Q| and P^T |dO| (fp64).
+    ``rows`` restricts the query rows (exact for those rows' dQ, and for the
+    dK / dV columns that only those rows reach)."""
     S = qg.shape[0]
     eq, ek, ev = np.zeros_like(qg), np.zeros_like(kg), np.zeros_like(vg)
     cols = np.arange(S)
-    for a in range(0, S, chunk):
-        r = np.arange(a, min(a + chunk, S))
+    rows = np.arange(S) if rows is None else np.asarray(rows, dtype=np.int64)
+    for a in range(0, rows.shape[0], chunk):
+        r = rows[a:a + chunk]
         s = (qg[r] @ kg.T) * scale
         s[cols[None, :] > r[:, None]] = -np.inf
         pr = np.exp(s - s.max(axis=1)[:, None])
