@@ -8,19 +8,18 @@
 // floating-point atomics, so every gradient is bitwise reproducible:
 //
 //  k_attn_bwd_dkdv  one CTA per 128 key rows of one (b, h); walks the query
-//                   tiles of 64 rows at and after its diagonal.  TMEM holds
-//                   S^T and dP^T (two buffers each, 64 columns) and the dV,
-//                   dK accumulators (d columns each).
+//                   tiles of 128 rows at and after its diagonal.  TMEM holds
+//                   S^T, dP^T (P^T, dS^T as bf16 in place) and the dV, dK
+//                   accumulators; the gradient MMAs read P^T / dS^T straight
+//                   from TMEM.  Two issuer warps (one per MMA stream).
 //  k_attn_bwd_dq    one CTA per 128 query rows; walks the key tiles of 64
 //                   rows up to its diagonal, recomputing S and dP, and
 //                   accumulates dQ in TMEM.
 //
-// Warp roles: warp 0 issues TMA loads (2-stage ring of the walked tiles),
-// warp 1 issues the MMAs from one thread and commits them to mbarriers, and
-// two softmax warpgroups (warps 2-9) own the TMEM lanes (= the rows of the
-// stationary tile), each warpgroup half of the walked tile's columns: they
-// turn scores into P and dS in fp32 and write them to shared memory as bf16
-// in the 128-byte-swizzled K-major layout the gradient MMAs read.  (The
+// Warp roles: warp 0 issues TMA loads of the walked tiles, MMA issuer warps
+// commit their MMAs to mbarriers, and two softmax warpgroups (8 warps) own
+// the TMEM lanes (= the rows of the stationary tile), each warpgroup half of
+// the walked tile's columns: they turn scores into P and dS in fp32.  (The
 // backward softmax is elementwise given LSE and D, so the two halves need no
 // exchange; two warps per SM sub-partition hide each other's latency.)
 // The same shared-memory tile of Q, dO or K serves as a K-major operand in
@@ -41,9 +40,12 @@ constexpr float kLog2e = 1.4426950408889634f;
 // ------------------------------------------------------------------ dK/dV --
 
 constexpr int KV_M = 128;  // stationary key rows
-constexpr int Q_N = 64;    // walked query rows per tile
+constexpr int Q_N = 128;   // walked query rows per tile
+constexpr int QST = 2;     // stages of the walked Q / dO ring
 
-constexpr int QST = 3;     // stages of the walked Q / dO ring
+// warp 0 TMA, warp 1 issuer A (S^T, dV), warps 2-9 softmax, warp 10 issuer B
+// (dP^T, dK).
+constexpr int kThreadsDkdv = 352;
 
 template <int HD>
 struct DkdvLayout {
@@ -51,23 +53,29 @@ struct DkdvLayout {
   static constexpr uint32_t v = k + KV_M * HD * 2;
   static constexpr uint32_t q = v + KV_M * HD * 2;            // QST stages
   static constexpr uint32_t dO = q + QST * Q_N * HD * 2;      // QST stages
-  static constexpr uint32_t p = dO + QST * Q_N * HD * 2;      // 2 x [128][64] bf16
-  static constexpr uint32_t ds = p + 2 * KV_M * Q_N * 2;      // 2 x [128][64] bf16
-  static constexpr uint32_t bar = ds + 2 * KV_M * Q_N * 2;
+  static constexpr uint32_t ld = dO + QST * Q_N * HD * 2;     // 2 x [LSE 128 | D 128] fp32
+  static constexpr uint32_t bar = ld + 2 * 2 * Q_N * 4;
   static constexpr uint32_t bytes = bar + 256;
 };
 
 struct DkdvBars {
-  // pfull is indexed by tile parity like the P/dS buffers: the softmax of
-  // tile i + 1 may finish before the issuer has seen tile i's phase, and a
-  // single barrier would then complete twice and hide phase i from it.
-  uint64_t kvfull, qfull[QST], qempty[QST], sfull[2], sfree[2], pfull[2], dsfree[2], done;
+  uint64_t kvfull, qfull[QST], qempty[QST], sfull, dpfull, pready, dsready, done;
   uint32_t tmem_base;
 };
 
-// Columns: S^T buffers 0/64, dP^T buffers 128/192, dV 256, dK 256 + HD.
+// TMEM columns: S^T 0..127 (P^T as packed bf16 over the first 32 columns of
+// each warpgroup's 64), dP^T 128..255 (dS^T likewise), dV 256, dK 256 + HD.
+//
+// Per query tile i the tensor pipe runs two independent streams, each from
+// its own issuer warp so that a barrier wait in one never drains the pipe:
+//   A: dV += P^T(i-1) dO(i-1), then S^T(i) = K Q(i)^T   (waits P(i-1))
+//   B: dK += dS^T(i-1) Q(i-1), then dP^T(i) = V dO(i)^T (waits dS(i-1))
+// The softmax warpgroups turn S^T(i) into P (fp32 in registers, bf16 into
+// TMEM) while stream B runs, then dP^T(i) into dS while stream A runs.  The
+// MMAs of one issuer execute in issue order, so S^T(i) overwriting P^T(i-1)
+// after the dV MMAs that read it is safe; likewise dP^T(i) after dK.
 template <int HD>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreadsDkdv, 1)
     k_attn_bwd_dkdv(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                     const float* __restrict__ lse, const float* __restrict__ delta,
@@ -82,22 +90,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kt = (int)(blockIdx.x / BH);  // key tile 0 walks the most query tiles: first
   const int bh = (int)(blockIdx.x % BH);
   const int n_q = (S + Q_N - 1) / Q_N;
-  const int i0 = kt * (KV_M / Q_N);  // first query tile at or after the diagonal
+  const int i0 = kt;                       // the diagonal query tile (Q_N == KV_M)
   const int n_it = n_q - i0;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kvfull, 1);
     for (int s = 0; s < QST; ++s) {
       mbar_init(&bars->qfull[s], 1);
-      mbar_init(&bars->qempty[s], 1);
+      mbar_init(&bars->qempty[s], 2);   // one commit from each issuer
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars->sfull[s], 1);
-      mbar_init(&bars->sfree[s], kSoftmax);
-      mbar_init(&bars->dsfree[s], 1);
-      mbar_init(&bars->pfull[s], kSoftmax);
-    }
-    mbar_init(&bars->done, 1);
+    mbar_init(&bars->sfull, 1);
+    mbar_init(&bars->dpfull, 1);
+    mbar_init(&bars->pready, kSoftmax);
+    mbar_init(&bars->dsready, kSoftmax);
+    mbar_init(&bars->done, 2);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -129,135 +135,141 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16(KV_M, Q_N, 0, 0);   // S^T, dP^T
-      constexpr uint32_t idG = idesc_bf16(KV_M, HD, 0, 1);    // dV, dK (B MN-major)
-      const uint32_t sK = smem_u32(smem + Lay::k), sV = smem_u32(smem + Lay::v);
-      const uint32_t sQ = smem_u32(smem + Lay::q), sO = smem_u32(smem + Lay::dO);
-      const uint32_t sP = smem_u32(smem + Lay::p), sDS = smem_u32(smem + Lay::ds);
-      bool ok = mbar_wait(&bars->kvfull, 0, status, 22);
-      auto grads = [&](int it) -> bool {
-        const int s = it % QST, pb = it & 1;
-        if (!mbar_wait(&bars->pfull[pb], (it >> 1) & 1, status, 23)) return false;
+  } else if (warp == 1 || warp == 10) {
+    // Issuer A (warp 1): S^T = K Q^T and dV += P^T dO.  Issuer B (warp 10):
+    // dP^T = V dO^T and dK += dS^T Q.  Whole-warp loops, one lane issues.
+    const bool isA = warp == 1;
+    constexpr uint32_t idS = idesc_bf16(KV_M, Q_N, 0, 0);   // S^T, dP^T
+    constexpr uint32_t idG = idesc_bf16(KV_M, HD, 0, 1);    // dV, dK (B MN-major)
+    const uint32_t sA = smem_u32(smem + (isA ? Lay::k : Lay::v));         // K or V
+    const uint32_t sB = smem_u32(smem + (isA ? Lay::q : Lay::dO));        // Q or dO ring
+    const uint32_t sG = smem_u32(smem + (isA ? Lay::dO : Lay::q));        // dO or Q ring
+    const uint32_t dSc = tmem + (isA ? 0u : 128u);                        // S^T or dP^T
+    const uint32_t dAcc = tmem + 256 + (isA ? 0u : (uint32_t)HD);         // dV or dK
+    uint64_t* ready = isA ? &bars->pready : &bars->dsready;
+    uint64_t* full = isA ? &bars->sfull : &bars->dpfull;
+    bool ok = mbar_wait_w(&bars->kvfull, 0, status, 22);
+    for (int it = 0; ok && it <= n_it; ++it) {
+      if (it > 0) {
+        // gradient MMAs of tile it - 1: A operand = P^T / dS^T (bf16 in TMEM)
+        const int sp = (it - 1) % QST;
+        if (!mbar_wait_w(ready, (it - 1) & 1, status, isA ? 23 : 24)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t qb = sQ + s * Q_N * HD * 2, ob = sO + s * Q_N * HD * 2;
+        const uint32_t gb = sG + sp * Q_N * HD * 2;
 #pragma unroll
-        for (int ks = 0; ks < Q_N / 16; ++ks) {
-          const uint64_t ap = sdesc_sw128(sP + pb * KV_M * Q_N * 2 + ks * 32, 16, 1024);
-          const uint64_t ad = sdesc_sw128(sDS + pb * KV_M * Q_N * 2 + ks * 32, 16, 1024);
-          const uint64_t bo = sdesc_sw128(ob + ks * 16 * 128, Q_N * 128, 1024);
-          const uint64_t bq = sdesc_sw128(qb + ks * 16 * 128, Q_N * 128, 1024);
-          const uint32_t acc = (it > 0 || ks > 0) ? 1u : 0u;
-          mma_bf16(tmem + 256, ap, bo, idG, acc);       // dV += P^T dO
-          mma_bf16(tmem + 256 + HD, ad, bq, idG, acc);  // dK += dS^T Q
-        }
-        mma_commit(&bars->dsfree[pb]);
-        mma_commit(&bars->qempty[s]);
-        return true;
-      };
-      for (int it = 0; ok && it < n_it; ++it) {
-        const int s = it % QST, sb = it & 1;
-        if (!mbar_wait(&bars->qfull[s], (it / QST) & 1, status, 24)) { ok = false; break; }
-        if (!mbar_wait(&bars->sfree[sb], ((it >> 1) & 1) ^ 1, status, 25)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t qb = sQ + s * Q_N * HD * 2, ob = sO + s * Q_N * HD * 2;
-#pragma unroll
-        for (int ks = 0; ks < HD / 16; ++ks) {
-          const uint32_t koff = (ks >> 2) * KV_M * 128 + (ks & 3) * 32;
-          const uint32_t qoff = (ks >> 2) * Q_N * 128 + (ks & 3) * 32;
-          mma_bf16(tmem + sb * Q_N, sdesc_sw128(sK + koff, 16, 1024),
-                   sdesc_sw128(qb + qoff, 16, 1024), idS, ks > 0 ? 1u : 0u);
-          mma_bf16(tmem + 128 + sb * Q_N, sdesc_sw128(sV + koff, 16, 1024),
-                   sdesc_sw128(ob + qoff, 16, 1024), idS, ks > 0 ? 1u : 0u);
-        }
-        mma_commit(&bars->sfull[sb]);
-        if (it > 0 && !grads(it - 1)) { ok = false; break; }
+        for (int ks = 0; ks < Q_N / 16; ++ks)
+          mma_bf16_ts_w(dAcc, dSc + (ks >> 2) * 64 + (ks & 3) * 8,
+                        sdesc_sw128(gb + ks * 16 * 128, Q_N * 128, 1024), idG,
+                        (it > 1 || ks > 0) ? 1u : 0u);
+        mma_commit_w(&bars->qempty[sp]);
       }
-      if (ok && grads(n_it - 1)) mma_commit(&bars->done);
+      if (it == n_it) break;
+      const int s = it % QST;
+      if (!mbar_wait_w(&bars->qfull[s], (it / QST) & 1, status, isA ? 25 : 26)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t bb = sB + s * Q_N * HD * 2;
+#pragma unroll
+      for (int ks = 0; ks < HD / 16; ++ks) {
+        const uint32_t aoff = (ks >> 2) * KV_M * 128 + (ks & 3) * 32;
+        const uint32_t boff = (ks >> 2) * Q_N * 128 + (ks & 3) * 32;
+        mma_bf16_w(dSc, sdesc_sw128(sA + aoff, 16, 1024), sdesc_sw128(bb + boff, 16, 1024), idS,
+                   ks > 0 ? 1u : 0u);
+      }
+      mma_commit_w(full);
     }
+    if (ok) mma_commit_w(&bars->done);
   } else {
+    // Softmax warpgroups: warp w owns TMEM lanes 32 (w % 4) .. +31 (key rows)
+    // and query columns 64 h .. 64 h + 63 of each tile, h = (w - 2) / 4.
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;                // which 32 of the 64 query columns
-    const int r = quarter * 32 + lane;               // key row in the tile
+    const int h = (warp - 2) >> 2;
+    const int r = quarter * 32 + lane;
     const int kvrow = kt * KV_M + r;
+    const int ts = threadIdx.x - 64;                 // 0..255 among the softmax threads
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-    uint8_t* pP = smem + Lay::p;
-    uint8_t* pDS = smem + Lay::ds;
+    const uint32_t cS = tmem + lane_addr + h * 64, cP = tmem + lane_addr + 128 + h * 64;
+    float* ldbuf = reinterpret_cast<float*>(smem + Lay::ld);
     const float c = scale * kLog2e;
-    const int c0 = half * 32;
+    // LSE (log2 units) or D of one query column per thread, staged in shared
+    // memory per tile: rows past S get LSE = +inf (P = 0) and D = 0.
+    auto ld_col = [&](int it) -> float {
+      const int q = (i0 + it) * Q_N + (ts & (Q_N - 1));
+      if (ts < Q_N) return q < S ? __ldg(lse + (int64_t)bh * S + q) * kLog2e : INFINITY;
+      return q < S ? __ldg(delta + (int64_t)bh * S + q) : 0.f;
+    };
+    ldbuf[ts] = ld_col(0);
+    named_bar(1, kSoftmax);
+    // After a failed wait a thread skips the work but keeps taking every
+    // named barrier, so the others never block on it.
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
-      const int sb = it & 1;
-      const int q0 = (i0 + it) * Q_N;
-      // LSE (log2 units) and D of this thread's 32 query columns; the
-      // addresses are the same across the warp, so each load is one request
-      // served from L1.  Rows past S get LSE = +inf (P = 0) and D = 0.
-      float lv[32], dv[32];
-      const int qb0 = q0 + c0;
-      const float* lrow = lse + (int64_t)bh * S + qb0;
-      const float* drow = delta + (int64_t)bh * S + qb0;
-      if (qb0 + 32 <= S) {
+      const float* lb = ldbuf + (it & 1) * 2 * Q_N;
+      const float nxt = (it + 1 < n_it) ? ld_col(it + 1) : 0.f;
+      const int qc0 = (i0 + it) * Q_N + h * 64;      // first query column of this thread
+      const bool diag = it == 0;
+      // ---- P = exp2(c s - lse): fp32 kept in registers, bf16 into TMEM
+      float p[64];
+      ok = ok && mbar_wait(&bars->sfull, it & 1, status, 27);
+      if (ok) {
+        tc_fence_after();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          lv[e] = __ldg(lrow + e) * kLog2e;
-          dv[e] = __ldg(drow + e);
-        }
-      } else {
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t sr[16];
+          tmem_ld16(cS + ch * 16, sr);
+          tmem_ld_wait();
+          uint32_t pk[8];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const bool in = qb0 + e < S;
-          lv[e] = in ? __ldg(lrow + e) * kLog2e : INFINITY;
-          dv[e] = in ? __ldg(drow + e) : 0.f;
+          for (int e = 0; e < 16; e += 4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(lb + h * 64 + ch * 16 + e);
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              float pv = ex2(fmaf(__uint_as_float(sr[e + u]), c, -lv[u]));
+              if (diag) pv = (qc0 + ch * 16 + e + u >= kvrow) ? pv : 0.f;
+              p[ch * 16 + e + u] = pv;
+            }
+            pk[e >> 1] = pack_bf16x2(p[ch * 16 + e], p[ch * 16 + e + 1]);
+            pk[(e >> 1) + 1] = pack_bf16x2(p[ch * 16 + e + 2], p[ch * 16 + e + 3]);
+          }
+          tmem_st8(cS + ch * 8, pk);
         }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bars->pready);
       }
-      if (!mbar_wait(&bars->sfull[sb], (it >> 1) & 1, status, 26)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t sr[32], pr[32];
-      tmem_ld32(tmem + lane_addr + sb * Q_N + c0, sr);
-      tmem_ld32(tmem + lane_addr + 128 + sb * Q_N + c0, pr);
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&bars->sfree[sb]);
-      uint32_t pk[16], dk[16];
-      if (q0 < kt * KV_M + KV_M) {                    // the tile crosses the diagonal
+      // ---- dS = P (dP - D), bf16 into TMEM
+      ok = ok && mbar_wait(&bars->dpfull, it & 1, status, 28);
+      if (ok) {
+        tc_fence_after();
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float p0 = ex2(fmaf(__uint_as_float(sr[e]), c, -lv[e]));
-          float p1 = ex2(fmaf(__uint_as_float(sr[e + 1]), c, -lv[e + 1]));
-          p0 = (q0 + c0 + e >= kvrow) ? p0 : 0.f;
-          p1 = (q0 + c0 + e + 1 >= kvrow) ? p1 : 0.f;
-          pk[e >> 1] = pack_bf16x2(p0, p1);
-          dk[e >> 1] = pack_bf16x2(p0 * (__uint_as_float(pr[e]) - dv[e]),
-                                   p1 * (__uint_as_float(pr[e + 1]) - dv[e + 1]));
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t pr[16];
+          tmem_ld16(cP + ch * 16, pr);
+          tmem_ld_wait();
+          uint32_t dk[8];
+#pragma unroll
+          for (int e = 0; e < 16; e += 4) {
+            const float4 d4 = *reinterpret_cast<const float4*>(lb + Q_N + h * 64 + ch * 16 + e);
+            dk[e >> 1] = pack_bf16x2(p[ch * 16 + e] * (__uint_as_float(pr[e]) - d4.x),
+                                     p[ch * 16 + e + 1] * (__uint_as_float(pr[e + 1]) - d4.y));
+            dk[(e >> 1) + 1] = pack_bf16x2(p[ch * 16 + e + 2] * (__uint_as_float(pr[e + 2]) - d4.z),
+                                           p[ch * 16 + e + 3] * (__uint_as_float(pr[e + 3]) - d4.w));
+          }
+          tmem_st8(cP + ch * 8, dk);
         }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const float p0 = ex2(fmaf(__uint_as_float(sr[e]), c, -lv[e]));
-          const float p1 = ex2(fmaf(__uint_as_float(sr[e + 1]), c, -lv[e + 1]));
-          pk[e >> 1] = pack_bf16x2(p0, p1);
-          dk[e >> 1] = pack_bf16x2(p0 * (__uint_as_float(pr[e]) - dv[e]),
-                                   p1 * (__uint_as_float(pr[e + 1]) - dv[e + 1]));
-        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bars->dsready);
       }
-      // P / dS buffer it % 2 was last read by the gradient MMAs of tile it - 2
-      const int pb = it & 1;
-      if (it >= 2 && !mbar_wait(&bars->dsfree[pb], ((it >> 1) & 1) ^ 1, status, 27)) { ok = false; break; }
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int cc = half * 4 + q;
-        const uint32_t off = pb * KV_M * Q_N * 2 + r * 128 + ((cc ^ (r & 7)) << 4);
-        *reinterpret_cast<uint4*>(pP + off) = make_uint4(pk[q * 4], pk[q * 4 + 1], pk[q * 4 + 2], pk[q * 4 + 3]);
-        *reinterpret_cast<uint4*>(pDS + off) = make_uint4(dk[q * 4], dk[q * 4 + 1], dk[q * 4 + 2], dk[q * 4 + 3]);
+      // ---- stage the next tile's LSE / D (its buffer was last read one tile ago)
+      if (it + 1 < n_it) {
+        ldbuf[((it + 1) & 1) * 2 * Q_N + ts] = nxt;
+        named_bar(1, kSoftmax);
       }
-      fence_async_smem();
-      tc_fence_before();
-      mbar_arrive(&bars->pfull[pb]);
     }
-    if (ok && mbar_wait(&bars->done, 0, status, 28)) {
+    if (ok && mbar_wait(&bars->done, 0, status, 29)) {
       tc_fence_after();
-      const int which = half;                        // warpgroup 0 writes dV, 1 writes dK
+      const int which = h;                           // warpgroup 0 writes dV, 1 writes dK
       uint4* dst = (which ? dkg : dvg) + ((int64_t)bh * S + kvrow) * (HD / 8);
       const float mul = which ? scale : 1.f;
 #pragma unroll
@@ -509,8 +521,8 @@ cudaError_t launch_hd(int BH, int S, float scale, const CUtensorMap* maps_q, con
   if (which & 1) {
     cudaFuncSetAttribute(k_attn_bwd_dkdv<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemDkdv);
     const int n_kt = (S + KV_M - 1) / KV_M;
-    k_attn_bwd_dkdv<HD><<<n_kt * BH, kThreads, kSmemDkdv, st>>>(
-        maps_q[0], maps_kv[1], maps_kv[2], maps_q[3], lse, delta, (uint4*)dkg, (uint4*)dvg, S, BH,
+    k_attn_bwd_dkdv<HD><<<n_kt * BH, kThreadsDkdv, kSmemDkdv, st>>>(
+        maps_kv[0], maps_kv[1], maps_kv[2], maps_kv[3], lse, delta, (uint4*)dkg, (uint4*)dvg, S, BH,
         scale, status);
   }
   if (which & 2) {
