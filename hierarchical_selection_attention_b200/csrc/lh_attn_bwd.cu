@@ -53,18 +53,35 @@ struct DkdvLayout {
   static constexpr uint32_t v = k + KV_M * HD * 2;
   static constexpr uint32_t q = v + KV_M * HD * 2;            // QST stages
   static constexpr uint32_t dO = q + QST * Q_N * HD * 2;      // QST stages
-  static constexpr uint32_t ld = dO + QST * Q_N * HD * 2;     // 2 x [LSE 128 | D 128] fp32
-  static constexpr uint32_t bar = ld + 2 * 2 * Q_N * 4;
+  static constexpr uint32_t kaug = dO + QST * Q_N * HD * 2;   // [128][16] bf16, constant
+  static constexpr uint32_t qaug = kaug + KV_M * 32;          // QST x [128][16] bf16
+  static constexpr uint32_t oaug = qaug + QST * Q_N * 32;     // QST x [128][16] bf16
+  static constexpr uint32_t bar = oaug + QST * Q_N * 32;
   static constexpr uint32_t bytes = bar + 256;
 };
 
 struct DkdvBars {
-  uint64_t kvfull, qfull[QST], qempty[QST], sfull, dpfull, pready, dsready, done;
+  // sissued[t % 2]: issuer A has issued S^T(t).  Issuer B waits for it before
+  // its own MMAs of step t, so the MMAs on the softmax's critical chain (dV,
+  // then S^T) enter the tensor pipe first.  Two barriers by parity, because
+  // A may run one step ahead of B.
+  uint64_t kvfull, qfull[QST], qempty[QST], sfull, dpfull, pready, dsready, sissued[2], done;
   uint32_t tmem_base;
 };
 
 // TMEM columns: S^T 0..127 (P^T as packed bf16 over the first 32 columns of
 // each warpgroup's 64), dP^T 128..255 (dS^T likewise), dV 256, dK 256 + HD.
+//
+// LSE and D enter through the tensor core, not through the softmax threads:
+// each score MMA gets one more K = 16 step whose A rows are (-1/2, -1/2,
+// -1/2, 0, ...) and whose B row for query q holds x_q split into three bf16
+// terms (hi + mid + lo = x_q to fp32 precision), both halves of every 32-byte
+// row equal, so the extra step adds -x_q exactly (products of bf16 are exact
+// in the fp32 accumulator).  With x = LSE / scale the first MMA yields
+// s - LSE / scale, so P = exp2(scale log2(e) (s - LSE / scale)); with x = D
+// the second yields dP - D.  The softmax threads then read nothing but TMEM:
+// shared-memory loads from those threads stall behind the tensor core's
+// operand reads.
 //
 // Per query tile i the tensor pipe runs two independent streams, each from
 // its own issuer warp so that a barrier wait in one never drains the pipe:
@@ -103,8 +120,15 @@ __global__ void __launch_bounds__(kThreadsDkdv, 1)
     mbar_init(&bars->dpfull, 1);
     mbar_init(&bars->pready, kSoftmax);
     mbar_init(&bars->dsready, kSoftmax);
+    mbar_init(&bars->sissued[0], 1);
+    mbar_init(&bars->sissued[1], 1);
     mbar_init(&bars->done, 2);
     fence_mbar_init();
+  }
+  if (threadIdx.x < 2 * KV_M) {                      // the constant A rows of the extra step
+    const uint32_t mh = pack_bf16x2(-0.5f, -0.5f), m0 = pack_bf16x2(-0.5f, 0.f);
+    *reinterpret_cast<uint4*>(smem + Lay::kaug + threadIdx.x * 16) = make_uint4(mh, m0, 0u, 0u);
+    fence_async_smem();
   }
   if (warp == 1) {
     tmem_alloc(&bars->tmem_base, kTmemCols);
@@ -116,15 +140,56 @@ __global__ void __launch_bounds__(kThreadsDkdv, 1)
   const uint32_t tmem = bars->tmem_base;
 
   if (warp == 0) {
+    // Producer warp: lane 0 issues the TMA loads; all lanes build the B rows
+    // of the extra K step for each query tile (rows lane + 32 j).
     if (lane == 0) {
       mbar_expect_tx(&bars->kvfull, 2 * KV_M * HD * 2);
       for (int blk = 0; blk < HD / 64; ++blk) {
         tma_load_3d(&tmK, &bars->kvfull, smem + Lay::k + blk * KV_M * 128, 64 * blk, kt * KV_M, bh);
         tma_load_3d(&tmV, &bars->kvfull, smem + Lay::v + blk * KV_M * 128, 64 * blk, kt * KV_M, bh);
       }
-      for (int it = 0; it < n_it; ++it) {
-        const int s = it % QST;
-        if (!mbar_wait(&bars->qempty[s], ((it / QST) & 1) ^ 1, status, 21)) break;
+    }
+    const float inv_scale = 1.f / scale;
+    float ln[4], dn[4];                              // next tile's LSE / D, rows past S: 0
+    auto fetch = [&](int it) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int q = (i0 + it) * Q_N + lane + 32 * j;
+        ln[j] = q < S ? __ldg(lse + (int64_t)bh * S + q) * inv_scale : 0.f;
+        dn[j] = q < S ? __ldg(delta + (int64_t)bh * S + q) : 0.f;
+      }
+    };
+    // x -> (hi, mid, lo) bf16 with hi + mid + lo = x to fp32 precision, as one
+    // 16-byte half row (hi, mid, lo, 0, 0, 0, 0, 0)
+    auto split3 = [](float x) -> uint4 {
+      const uint32_t h2 = pack_bf16x2(x, 0.f);
+      const float r1 = x - __uint_as_float(h2 << 16);
+      const uint32_t m2 = pack_bf16x2(r1, 0.f);
+      const float r2 = r1 - __uint_as_float(m2 << 16);
+      return make_uint4((h2 & 0xffffu) | (m2 << 16), pack_bf16x2(r2, 0.f), 0u, 0u);
+    };
+    fetch(0);
+    for (int it = 0; it < n_it; ++it) {
+      const int s = it % QST;
+      float lc[4], dc[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) { lc[j] = ln[j]; dc[j] = dn[j]; }
+      if (it + 1 < n_it) fetch(it + 1);
+      if (!mbar_wait_w(&bars->qempty[s], ((it / QST) & 1) ^ 1, status, 21)) break;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int r = lane + 32 * j;
+        const uint4 wl = split3(lc[j]), wd = split3(dc[j]);
+        uint8_t* ql = smem + Lay::qaug + s * Q_N * 32 + r * 32;
+        uint8_t* ol = smem + Lay::oaug + s * Q_N * 32 + r * 32;
+        *reinterpret_cast<uint4*>(ql) = wl;
+        *reinterpret_cast<uint4*>(ql + 16) = wl;
+        *reinterpret_cast<uint4*>(ol) = wd;
+        *reinterpret_cast<uint4*>(ol + 16) = wd;
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) {
         mbar_expect_tx(&bars->qfull[s], 2 * Q_N * HD * 2);
         const int row = (i0 + it) * Q_N;
         for (int blk = 0; blk < HD / 64; ++blk) {
@@ -134,6 +199,7 @@ __global__ void __launch_bounds__(kThreadsDkdv, 1)
                       64 * blk, row, bh);
         }
       }
+      __syncwarp();
     }
   } else if (warp == 1 || warp == 10) {
     // Issuer A (warp 1): S^T = K Q^T and dV += P^T dO.  Issuer B (warp 10):
@@ -142,6 +208,8 @@ __global__ void __launch_bounds__(kThreadsDkdv, 1)
     constexpr uint32_t idS = idesc_bf16(KV_M, Q_N, 0, 0);   // S^T, dP^T
     constexpr uint32_t idG = idesc_bf16(KV_M, HD, 0, 1);    // dV, dK (B MN-major)
     const uint32_t sA = smem_u32(smem + (isA ? Lay::k : Lay::v));         // K or V
+    const uint32_t sKaug = smem_u32(smem + Lay::kaug);
+    const uint32_t sBaug = smem_u32(smem + (isA ? Lay::qaug : Lay::oaug)); // -LSE/scale or -D
     const uint32_t sB = smem_u32(smem + (isA ? Lay::q : Lay::dO));        // Q or dO ring
     const uint32_t sG = smem_u32(smem + (isA ? Lay::dO : Lay::q));        // dO or Q ring
     const uint32_t dSc = tmem + (isA ? 0u : 128u);                        // S^T or dP^T
@@ -150,6 +218,8 @@ __global__ void __launch_bounds__(kThreadsDkdv, 1)
     uint64_t* full = isA ? &bars->sfull : &bars->dpfull;
     bool ok = mbar_wait_w(&bars->kvfull, 0, status, 22);
     for (int it = 0; ok && it <= n_it; ++it) {
+      if (!isA && it < n_it &&
+          !mbar_wait_w(&bars->sissued[it & 1], (it >> 1) & 1, status, 20)) { ok = false; break; }
       if (it > 0) {
         // gradient MMAs of tile it - 1: A operand = P^T / dS^T (bf16 in TMEM)
         const int sp = (it - 1) % QST;
@@ -175,7 +245,9 @@ __global__ void __launch_bounds__(kThreadsDkdv, 1)
         mma_bf16_w(dSc, sdesc_sw128(sA + aoff, 16, 1024), sdesc_sw128(bb + boff, 16, 1024), idS,
                    ks > 0 ? 1u : 0u);
       }
+      mma_bf16_w(dSc, sdesc_sw32(sKaug), sdesc_sw32(sBaug + s * Q_N * 32), idS, 1u);
       mma_commit_w(full);
+      if (isA && lane == 0) mbar_arrive(&bars->sissued[it & 1]);
     }
     if (ok) mma_commit_w(&bars->done);
   } else {
@@ -185,87 +257,69 @@ __global__ void __launch_bounds__(kThreadsDkdv, 1)
     const int h = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;
     const int kvrow = kt * KV_M + r;
-    const int ts = threadIdx.x - 64;                 // 0..255 among the softmax threads
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
     const uint32_t cS = tmem + lane_addr + h * 64, cP = tmem + lane_addr + 128 + h * 64;
-    float* ldbuf = reinterpret_cast<float*>(smem + Lay::ld);
     const float c = scale * kLog2e;
-    // LSE (log2 units) or D of one query column per thread, staged in shared
-    // memory per tile: rows past S get LSE = +inf (P = 0) and D = 0.
-    auto ld_col = [&](int it) -> float {
-      const int q = (i0 + it) * Q_N + (ts & (Q_N - 1));
-      if (ts < Q_N) return q < S ? __ldg(lse + (int64_t)bh * S + q) * kLog2e : INFINITY;
-      return q < S ? __ldg(delta + (int64_t)bh * S + q) : 0.f;
-    };
-    ldbuf[ts] = ld_col(0);
-    named_bar(1, kSoftmax);
-    // After a failed wait a thread skips the work but keeps taking every
-    // named barrier, so the others never block on it.
     bool ok = true;
-    for (int it = 0; it < n_it; ++it) {
-      const float* lb = ldbuf + (it & 1) * 2 * Q_N;
-      const float nxt = (it + 1 < n_it) ? ld_col(it + 1) : 0.f;
+    for (int it = 0; ok && it < n_it; ++it) {
       const int qc0 = (i0 + it) * Q_N + h * 64;      // first query column of this thread
       const bool diag = it == 0;
-      // ---- P = exp2(c s - lse): fp32 kept in registers, bf16 into TMEM
-      float p[64];
-      ok = ok && mbar_wait(&bars->sfull, it & 1, status, 27);
-      if (ok) {
-        tc_fence_after();
+      // ---- P = exp2(c (s - LSE / scale)): fp32 kept in registers, bf16 into TMEM
+      uint32_t p[64];                                // scores, then P (fp32 bits)
+      if (!mbar_wait(&bars->sfull, it & 1, status, 27)) { ok = false; break; }
+      tc_fence_after();
+      tmem_ld32(cS, *reinterpret_cast<uint32_t(*)[32]>(&p[0]));
+      tmem_ld32(cS + 32, *reinterpret_cast<uint32_t(*)[32]>(&p[32]));
+      tmem_ld_wait();
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t sr[16];
-          tmem_ld16(cS + ch * 16, sr);
-          tmem_ld_wait();
-          uint32_t pk[8];
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t pk[8];
 #pragma unroll
-          for (int e = 0; e < 16; e += 4) {
-            const float4 l4 = *reinterpret_cast<const float4*>(lb + h * 64 + ch * 16 + e);
-            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              float pv = ex2(fmaf(__uint_as_float(sr[e + u]), c, -lv[u]));
-              if (diag) pv = (qc0 + ch * 16 + e + u >= kvrow) ? pv : 0.f;
-              p[ch * 16 + e + u] = pv;
-            }
-            pk[e >> 1] = pack_bf16x2(p[ch * 16 + e], p[ch * 16 + e + 1]);
-            pk[(e >> 1) + 1] = pack_bf16x2(p[ch * 16 + e + 2], p[ch * 16 + e + 3]);
+        for (int e = 0; e < 16; e += 2) {
+          const int j = ch * 16 + e;
+          const float x0 = __uint_as_float(p[j]) * c, x1 = __uint_as_float(p[j + 1]) * c;
+          float p0 = ex2(x0);
+          float p1 = ex2(x1);
+          if (diag) {
+            p0 = (qc0 + j >= kvrow) ? p0 : 0.f;
+            p1 = (qc0 + j + 1 >= kvrow) ? p1 : 0.f;
           }
-          tmem_st8(cS + ch * 8, pk);
+          p[j] = __float_as_uint(p0);
+          p[j + 1] = __float_as_uint(p1);
+          pk[e >> 1] = pack_bf16x2(p0, p1);
         }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&bars->pready);
+        // packed P of columns 16 ch .. 16 ch + 15 lands on fp32 columns
+        // 8 ch .. 8 ch + 7 of this thread's range, already read above
+        tmem_st8(cS + ch * 8, pk);
       }
-      // ---- dS = P (dP - D), bf16 into TMEM
-      ok = ok && mbar_wait(&bars->dpfull, it & 1, status, 28);
-      if (ok) {
-        tc_fence_after();
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars->pready);
+      // ---- dS = P (dP - D), bf16 into TMEM; the dP loads run one chunk ahead
+      if (!mbar_wait(&bars->dpfull, it & 1, status, 28)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t pr[2][16];
+      tmem_ld16(cP, pr[0]);
+      tmem_ld_wait();
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t pr[16];
-          tmem_ld16(cP + ch * 16, pr);
-          tmem_ld_wait();
-          uint32_t dk[8];
+      for (int ch = 0; ch < 4; ++ch) {
+        if (ch < 3) tmem_ld16(cP + (ch + 1) * 16, pr[(ch + 1) & 1]);
+        const uint32_t* q = pr[ch & 1];
+        uint32_t dk[8];
 #pragma unroll
-          for (int e = 0; e < 16; e += 4) {
-            const float4 d4 = *reinterpret_cast<const float4*>(lb + Q_N + h * 64 + ch * 16 + e);
-            dk[e >> 1] = pack_bf16x2(p[ch * 16 + e] * (__uint_as_float(pr[e]) - d4.x),
-                                     p[ch * 16 + e + 1] * (__uint_as_float(pr[e + 1]) - d4.y));
-            dk[(e >> 1) + 1] = pack_bf16x2(p[ch * 16 + e + 2] * (__uint_as_float(pr[e + 2]) - d4.z),
-                                           p[ch * 16 + e + 3] * (__uint_as_float(pr[e + 3]) - d4.w));
-          }
-          tmem_st8(cP + ch * 8, dk);
+        for (int e = 0; e < 16; e += 2) {
+          const int j = ch * 16 + e;
+          dk[e >> 1] = pack_bf16x2(__uint_as_float(p[j]) * __uint_as_float(q[e]),
+                                   __uint_as_float(p[j + 1]) * __uint_as_float(q[e + 1]));
         }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&bars->dsready);
+        // chunk ch's packed dS covers fp32 columns 8 ch .. 8 ch + 7, all
+        // read by the loads of chunks <= ch, which have completed
+        tmem_st8(cP + ch * 8, dk);
+        if (ch < 3) tmem_ld_wait();
       }
-      // ---- stage the next tile's LSE / D (its buffer was last read one tile ago)
-      if (it + 1 < n_it) {
-        ldbuf[((it + 1) & 1) * 2 * Q_N + ts] = nxt;
-        named_bar(1, kSoftmax);
-      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars->dsready);
     }
     if (ok && mbar_wait(&bars->done, 0, status, 29)) {
       tc_fence_after();

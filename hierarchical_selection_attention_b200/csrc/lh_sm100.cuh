@@ -215,6 +215,17 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
          (2ull << 61);                                                    // 128B swizzle
 }
 
+// Shared-memory matrix descriptor for a K-major operand of K = 16 bf16 per
+// row (32-byte rows) in the 32-byte-swizzled layout: 8-row atoms of 256
+// bytes, sbo = 256.  A row whose two 16-byte halves are equal reads the same
+// under any swizzle, which lets threads write such tiles without knowing
+// the swizzle pattern.
+__device__ __forceinline__ uint64_t sdesc_sw32(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) |
+         ((uint64_t)(256 >> 4) << 32) | (1ull << 46) |  // sm100 version
+         (6ull << 61);                                   // 32B swizzle
+}
+
 // 32 lanes x 32 columns of 32-bit words: thread i of the warp gets the 32
 // words of TMEM lane (warp quarter * 32 + i) starting at the column in taddr.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
@@ -281,6 +292,25 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x evaluated on the FMA pipe instead of the special-function unit, for
+// kernels whose exponentials saturate that unit (16 per clock per SM): the
+// caller sends a fraction of its elements here.  x = n + f with n the
+// nearest integer (rounded by adding 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f
+// by a degree-4 polynomial that interpolates 2^f at the five Chebyshev nodes
+// of [-1/2, 1/2] (coefficients from fit_exp2_poly.py beside this file,
+// maximum relative error 3.6e-6); 2^n is added into the exponent field.
+// Valid for -126 <= x < 128; smaller x is clamped to -126.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -126.f);
+  const float t = x + 12582912.f;
+  const float f = x - (t - 12582912.f);
+  float p = fmaf(0x1.3cbf60p-7f, f, 0x1.ca1ce2p-5f);
+  p = fmaf(p, f, 0x1.ebfa4cp-3f);
+  p = fmaf(p, f, 0x1.62e0c2p-1f);
+  p = fmaf(p, f, 1.0f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 // Named barrier over `nthreads` threads (multiple of 32) with id `id` (1..15).
