@@ -12,9 +12,10 @@
 //                   S^T, dP^T (P^T, dS^T as bf16 in place) and the dV, dK
 //                   accumulators; the gradient MMAs read P^T / dS^T straight
 //                   from TMEM.  Two issuer warps (one per MMA stream).
-//  k_attn_bwd_dq    one CTA per 128 query rows; walks the key tiles of 64
-//                   rows up to its diagonal, recomputing S and dP, and
-//                   accumulates dQ in TMEM.
+//  k_attn_bwd_dq    one CTA per 128 query rows; walks the key tiles of 128
+//                   rows up to its diagonal, recomputing S (two TMEM
+//                   buffers) and dP (dS as bf16 in place), and accumulates
+//                   dQ in TMEM from TS MMAs.  Two issuer warps.
 //
 // Warp roles: warp 0 issues TMA loads of the walked tiles, MMA issuer warps
 // commit their MMAs to mbarriers, and two softmax warpgroups (8 warps) own
@@ -30,9 +31,9 @@ namespace {
 
 using namespace sm100;
 
-// warp 0 TMA, warp 1 MMA, warps 2-9 two softmax warpgroups: warp w owns TMEM
-// lanes 32 (w % 4) .. +31 and half (w - 2) / 4 of the walked tile's columns.
-constexpr int kThreads = 320;
+// Both kernels: warp 0 TMA, warps 1 and 10 MMA issuers, warps 2-9 two
+// softmax warpgroups (warp w owns TMEM lanes 32 (w % 4) .. +31 and half
+// (w - 2) / 4 of the walked tile's columns).
 constexpr int kSoftmax = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -356,30 +357,45 @@ __global__ void __launch_bounds__(kThreadsDkdv, 1)
 // --------------------------------------------------------------------- dQ --
 
 constexpr int Q_M = 128;   // stationary query rows
-constexpr int KV_N = 64;   // walked key rows per tile
+constexpr int KV_N = 128;  // walked key rows per tile
+constexpr int KST = 3;     // stages of the walked K ring (K is held until the dQ MMAs)
+constexpr int VST = 2;     // stages of the walked V ring (V only until the dP MMAs)
 
-constexpr int KST = 4;     // stages of the walked K / V ring
+// warp 0 TMA, warp 1 issuer A (S), warps 2-9 softmax, warp 10 issuer B (dQ, dP)
+constexpr int kThreadsDq = 352;
 
 template <int HD>
 struct DqLayout {
   static constexpr uint32_t q = 0;
   static constexpr uint32_t dO = q + Q_M * HD * 2;
   static constexpr uint32_t k = dO + Q_M * HD * 2;          // KST stages
-  static constexpr uint32_t v = k + KST * KV_N * HD * 2;     // KST stages
-  static constexpr uint32_t bar = v + KST * KV_N * HD * 2;
+  static constexpr uint32_t v = k + KST * KV_N * HD * 2;     // VST stages
+  static constexpr uint32_t bar = v + VST * KV_N * HD * 2;
   static constexpr uint32_t bytes = bar + 256;
 };
 
 struct DqBars {
-  // pfull per tile parity, for the reason given at DkdvBars
-  uint64_t qfull, kvfull[KST], kvempty[KST], sfull[2], sfree[2], pfull[2], dsfree[2], done;
+  // dpissued[t % 2]: issuer B has issued dP(t).  Issuer A waits for it before
+  // S(t + 1), so B's MMAs (dQ, dP: the softmax's critical chain) enter the
+  // tensor pipe first and A's fill the time B waits for the softmax.  Two
+  // barriers by parity, because B may run one step ahead of A's wait.
+  uint64_t qfull, kfull[KST], kempty[KST], vfull[VST], vempty[VST], sfull[2], sfree[2], dpfull,
+      dsready, dpissued[2], done;
   uint32_t tmem_base;
 };
 
-// Columns: S buffers 0/64, dP buffers 128/192, dQ 256, dS (bf16 pairs)
-// buffers 384/416.
+// TMEM columns: S buffers 0 / 128, dP 256..383 (dS as packed bf16 over the
+// first 32 columns of each warpgroup's 64), dQ 384.
+//
+// Issuer A computes S(j) = Q K(j)^T into the S buffer j % 2 as soon as the
+// softmax has read S(j - 2); issuer B runs dQ += dS(j - 1) K(j - 1), then
+// dP(j) = dO V(j)^T (in issue order, so dP(j) overwrites dS(j - 1) only
+// after the dQ MMAs that read it).  The softmax turns S(j) into P in
+// registers while B's MMAs run, then dP(j) into dS.  LSE and D are
+// per-row values, so the softmax threads (one query row each) hold them in
+// registers and read nothing but TMEM in the loop.
 template <int HD>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreadsDq, 1)
     k_attn_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                   const float* __restrict__ lse, const float* __restrict__ delta,
@@ -393,20 +409,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_qt = (S + Q_M - 1) / Q_M;
   const int qt = n_qt - 1 - (int)(blockIdx.x / BH);  // longest rows first
   const int bh = (int)(blockIdx.x % BH);
-  const int n_kv = min((qt * Q_M + Q_M) / KV_N, (S + KV_N - 1) / KV_N);
+  const int n_kv = qt + 1;                           // key tiles up to the diagonal (KV_N == Q_M)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->qfull, 1);
     for (int s = 0; s < KST; ++s) {
-      mbar_init(&bars->kvfull[s], 1);
-      mbar_init(&bars->kvempty[s], 1);
+      mbar_init(&bars->kfull[s], 1);
+      mbar_init(&bars->kempty[s], 1);
+    }
+    for (int s = 0; s < VST; ++s) {
+      mbar_init(&bars->vfull[s], 1);
+      mbar_init(&bars->vempty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->sfull[s], 1);
       mbar_init(&bars->sfree[s], kSoftmax);
-      mbar_init(&bars->dsfree[s], 1);
-      mbar_init(&bars->pfull[s], kSoftmax);
     }
+    mbar_init(&bars->dpfull, 1);
+    mbar_init(&bars->dsready, kSoftmax);
+    mbar_init(&bars->dpissued[0], 1);
+    mbar_init(&bars->dpissued[1], 1);
     mbar_init(&bars->done, 1);
     fence_mbar_init();
   }
@@ -427,116 +449,147 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(&tmO, &bars->qfull, smem + Lay::dO + blk * Q_M * 128, 64 * blk, qt * Q_M, bh);
       }
       for (int j = 0; j < n_kv; ++j) {
-        const int s = j % KST;
-        if (!mbar_wait(&bars->kvempty[s], ((j / KST) & 1) ^ 1, status, 31)) break;
-        mbar_expect_tx(&bars->kvfull[s], 2 * KV_N * HD * 2);
-        for (int blk = 0; blk < HD / 64; ++blk) {
-          tma_load_3d(&tmK, &bars->kvfull[s], smem + Lay::k + s * KV_N * HD * 2 + blk * KV_N * 128,
+        const int s = j % KST, t = j % VST;
+        if (!mbar_wait(&bars->kempty[s], ((j / KST) & 1) ^ 1, status, 31)) break;
+        mbar_expect_tx(&bars->kfull[s], KV_N * HD * 2);
+        for (int blk = 0; blk < HD / 64; ++blk)
+          tma_load_3d(&tmK, &bars->kfull[s], smem + Lay::k + s * KV_N * HD * 2 + blk * KV_N * 128,
                       64 * blk, j * KV_N, bh);
-          tma_load_3d(&tmV, &bars->kvfull[s], smem + Lay::v + s * KV_N * HD * 2 + blk * KV_N * 128,
+        if (!mbar_wait(&bars->vempty[t], ((j / VST) & 1) ^ 1, status, 30)) break;
+        mbar_expect_tx(&bars->vfull[t], KV_N * HD * 2);
+        for (int blk = 0; blk < HD / 64; ++blk)
+          tma_load_3d(&tmV, &bars->vfull[t], smem + Lay::v + t * KV_N * HD * 2 + blk * KV_N * 128,
                       64 * blk, j * KV_N, bh);
-        }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16(Q_M, KV_N, 0, 0);   // S, dP
-      constexpr uint32_t idG = idesc_bf16(Q_M, HD, 0, 1);     // dQ (B = K, MN-major)
-      const uint32_t sQ = smem_u32(smem + Lay::q), sO = smem_u32(smem + Lay::dO);
-      const uint32_t sK = smem_u32(smem + Lay::k), sV = smem_u32(smem + Lay::v);
-      bool ok = mbar_wait(&bars->qfull, 0, status, 32);
-      auto grad = [&](int j) -> bool {
-        const int s = j % KST, pb = j & 1;
-        if (!mbar_wait(&bars->pfull[pb], (j >> 1) & 1, status, 33)) return false;
+    // Issuer A: S(j) = Q K(j)^T into buffer j % 2.  Whole-warp loop.
+    constexpr uint32_t idS = idesc_bf16(Q_M, KV_N, 0, 0);
+    const uint32_t sQ = smem_u32(smem + Lay::q), sK = smem_u32(smem + Lay::k);
+    bool ok = mbar_wait_w(&bars->qfull, 0, status, 32);
+    for (int j = 0; ok && j < n_kv; ++j) {
+      const int s = j % KST, sb = j & 1;
+      if (!mbar_wait_w(&bars->kfull[s], (j / KST) & 1, status, 33)) break;
+      if (!mbar_wait_w(&bars->sfree[sb], ((j >> 1) & 1) ^ 1, status, 34)) break;
+      if (j > 0 && !mbar_wait_w(&bars->dpissued[(j - 1) & 1], ((j - 1) >> 1) & 1, status, 29)) break;
+      tc_fence_after();
+      const uint32_t kb = sK + s * KV_N * HD * 2;
+#pragma unroll
+      for (int ks = 0; ks < HD / 16; ++ks) {
+        const uint32_t qoff = (ks >> 2) * Q_M * 128 + (ks & 3) * 32;
+        const uint32_t koff = (ks >> 2) * KV_N * 128 + (ks & 3) * 32;
+        mma_bf16_w(tmem + sb * KV_N, sdesc_sw128(sQ + qoff, 16, 1024),
+                   sdesc_sw128(kb + koff, 16, 1024), idS, ks > 0 ? 1u : 0u);
+      }
+      mma_commit_w(&bars->sfull[sb]);
+    }
+  } else if (warp == 10) {
+    // Issuer B: dQ += dS(j - 1) K(j - 1) (A operand from TMEM), then
+    // dP(j) = dO V(j)^T.  Whole-warp loop.
+    constexpr uint32_t idS = idesc_bf16(Q_M, KV_N, 0, 0);
+    constexpr uint32_t idG = idesc_bf16(Q_M, HD, 0, 1);     // dQ (B = K, MN-major)
+    const uint32_t sO = smem_u32(smem + Lay::dO), sK = smem_u32(smem + Lay::k);
+    const uint32_t sV = smem_u32(smem + Lay::v);
+    bool ok = mbar_wait_w(&bars->qfull, 0, status, 35);
+    for (int j = 0; ok && j <= n_kv; ++j) {
+      if (j > 0) {
+        const int sp = (j - 1) % KST;
+        if (!mbar_wait_w(&bars->dsready, (j - 1) & 1, status, 36)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t kb = sK + s * KV_N * HD * 2;
+        const uint32_t kb = sK + sp * KV_N * HD * 2;
 #pragma unroll
         for (int ks = 0; ks < KV_N / 16; ++ks)
-          mma_bf16_ts(tmem + 256, tmem + 384 + pb * 32 + ks * 8,
-                      sdesc_sw128(kb + ks * 16 * 128, KV_N * 128, 1024), idG,
-                      (j > 0 || ks > 0) ? 1u : 0u);
-        mma_commit(&bars->dsfree[pb]);
-        mma_commit(&bars->kvempty[s]);
-        return true;
-      };
-      for (int j = 0; ok && j < n_kv; ++j) {
-        const int s = j % KST, sb = j & 1;
-        if (!mbar_wait(&bars->kvfull[s], (j / KST) & 1, status, 34)) { ok = false; break; }
-        if (!mbar_wait(&bars->sfree[sb], ((j >> 1) & 1) ^ 1, status, 35)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t kb = sK + s * KV_N * HD * 2, vb = sV + s * KV_N * HD * 2;
-#pragma unroll
-        for (int ks = 0; ks < HD / 16; ++ks) {
-          const uint32_t qoff = (ks >> 2) * Q_M * 128 + (ks & 3) * 32;
-          const uint32_t koff = (ks >> 2) * KV_N * 128 + (ks & 3) * 32;
-          mma_bf16(tmem + sb * KV_N, sdesc_sw128(sQ + qoff, 16, 1024),
-                   sdesc_sw128(kb + koff, 16, 1024), idS, ks > 0 ? 1u : 0u);
-          mma_bf16(tmem + 128 + sb * KV_N, sdesc_sw128(sO + qoff, 16, 1024),
-                   sdesc_sw128(vb + koff, 16, 1024), idS, ks > 0 ? 1u : 0u);
-        }
-        mma_commit(&bars->sfull[sb]);
-        if (j > 0 && !grad(j - 1)) { ok = false; break; }
+          mma_bf16_ts_w(tmem + 384, tmem + 256 + (ks >> 2) * 64 + (ks & 3) * 8,
+                        sdesc_sw128(kb + ks * 16 * 128, KV_N * 128, 1024), idG,
+                        (j > 1 || ks > 0) ? 1u : 0u);
+        mma_commit_w(&bars->kempty[sp]);
       }
-      if (ok && grad(n_kv - 1)) mma_commit(&bars->done);
+      if (j == n_kv) break;
+      const int t = j % VST;
+      if (!mbar_wait_w(&bars->vfull[t], (j / VST) & 1, status, 37)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t vb = sV + t * KV_N * HD * 2;
+#pragma unroll
+      for (int ks = 0; ks < HD / 16; ++ks) {
+        const uint32_t qoff = (ks >> 2) * Q_M * 128 + (ks & 3) * 32;
+        const uint32_t koff = (ks >> 2) * KV_N * 128 + (ks & 3) * 32;
+        mma_bf16_w(tmem + 256, sdesc_sw128(sO + qoff, 16, 1024), sdesc_sw128(vb + koff, 16, 1024),
+                   idS, ks > 0 ? 1u : 0u);
+      }
+      mma_commit_w(&bars->dpfull);
+      mma_commit_w(&bars->vempty[t]);
+      if (lane == 0) mbar_arrive(&bars->dpissued[j & 1]);
     }
+    if (ok) mma_commit_w(&bars->done);
   } else {
+    // Softmax warpgroups: warp w owns TMEM lanes 32 (w % 4) .. +31 (query
+    // rows) and key columns 64 h .. 64 h + 63 of each tile, h = (w - 2) / 4.
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;                // which 32 of the 64 key columns
+    const int h = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;
     const int qrow = qt * Q_M + r;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+    const uint32_t cP = tmem + lane_addr + 256 + h * 64;
     const float c = scale * kLog2e;
-    const int c0 = half * 32;
     const float lrow = qrow < S ? __ldg(lse + (int64_t)bh * S + qrow) * kLog2e : INFINITY;
     const float drow = qrow < S ? __ldg(delta + (int64_t)bh * S + qrow) : 0.f;
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
+    for (int j = 0; ok && j < n_kv; ++j) {
       const int sb = j & 1;
-      const int k0 = j * KV_N;
-      if (!mbar_wait(&bars->sfull[sb], (j >> 1) & 1, status, 36)) { ok = false; break; }
+      const int kc0 = j * KV_N + h * 64;               // first key column of this thread
+      const bool diag = j == qt;
+      // ---- P = exp2(c s - lse), fp32 in registers
+      uint32_t p[64];
+      if (!mbar_wait(&bars->sfull[sb], (j >> 1) & 1, status, 38)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sr[32], pr[32];
-      tmem_ld32(tmem + lane_addr + sb * KV_N + c0, sr);
-      tmem_ld32(tmem + lane_addr + 128 + sb * KV_N + c0, pr);
+      const uint32_t cS = tmem + lane_addr + sb * KV_N + h * 64;
+      tmem_ld32(cS, *reinterpret_cast<uint32_t(*)[32]>(&p[0]));
+      tmem_ld32(cS + 32, *reinterpret_cast<uint32_t(*)[32]>(&p[32]));
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&bars->sfree[sb]);
-      uint32_t dk[16];
-      if (k0 + KV_N > qt * Q_M) {                     // the tile crosses the diagonal
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float p0 = ex2(fmaf(__uint_as_float(sr[e]), c, -lrow));
-          float p1 = ex2(fmaf(__uint_as_float(sr[e + 1]), c, -lrow));
-          p0 = (k0 + c0 + e <= qrow) ? p0 : 0.f;
-          p1 = (k0 + c0 + e + 1 <= qrow) ? p1 : 0.f;
-          dk[e >> 1] = pack_bf16x2(p0 * (__uint_as_float(pr[e]) - drow),
-                                   p1 * (__uint_as_float(pr[e + 1]) - drow));
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const float p0 = ex2(fmaf(__uint_as_float(sr[e]), c, -lrow));
-          const float p1 = ex2(fmaf(__uint_as_float(sr[e + 1]), c, -lrow));
-          dk[e >> 1] = pack_bf16x2(p0 * (__uint_as_float(pr[e]) - drow),
-                                   p1 * (__uint_as_float(pr[e + 1]) - drow));
-        }
+      for (int e = 0; e < 64; ++e) {
+        float pv = ex2(fmaf(__uint_as_float(p[e]), c, -lrow));
+        if (diag) pv = (kc0 + e <= qrow) ? pv : 0.f;
+        p[e] = __float_as_uint(pv);
       }
-      // dS buffer j % 2 (TMEM) was last read by the dQ MMAs of tile j - 2
-      const int pb = j & 1;
-      if (j >= 2 && !mbar_wait(&bars->dsfree[pb], ((j >> 1) & 1) ^ 1, status, 37)) { ok = false; break; }
-      tmem_st16(tmem + lane_addr + 384 + pb * 32 + half * 16, dk);
+#pragma unroll
+      for (int g = 0; g < 4; ++g) materialize16(p + 16 * g);
+      // ---- dS = P (dP - D), bf16 into TMEM; the dP loads run one chunk ahead
+      if (!mbar_wait(&bars->dpfull, j & 1, status, 39)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t pr[2][16];
+      tmem_ld16(cP, pr[0]);
+      tmem_ld_wait();
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        if (ch < 3) tmem_ld16(cP + (ch + 1) * 16, pr[(ch + 1) & 1]);
+        const uint32_t* q = pr[ch & 1];
+        uint32_t dk[8];
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {
+          const int i = ch * 16 + e;
+          dk[e >> 1] = pack_bf16x2(__uint_as_float(p[i]) * (__uint_as_float(q[e]) - drow),
+                                   __uint_as_float(p[i + 1]) * (__uint_as_float(q[e + 1]) - drow));
+        }
+        // chunk ch's packed dS covers fp32 columns 8 ch .. 8 ch + 7, all
+        // read by the loads of chunks <= ch, which have completed
+        tmem_st8(cP + ch * 8, dk);
+        if (ch < 3) tmem_ld_wait();
+      }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bars->pfull[pb]);
+      mbar_arrive(&bars->dsready);
     }
-    if (ok && mbar_wait(&bars->done, 0, status, 38)) {
+    if (ok && mbar_wait(&bars->done, 0, status, 40)) {
       tc_fence_after();
       uint4* dst = dqg + ((int64_t)bh * S + qrow) * (HD / 8);
 #pragma unroll
       for (int q = 0; q < HD / 64; ++q) {            // each warpgroup: half of the d columns
-        const int cchunk = half * (HD / 64) + q;
+        const int cchunk = h * (HD / 64) + q;
         uint32_t o[32];
-        tmem_ld32(tmem + lane_addr + 256 + cchunk * 32, o);
+        tmem_ld32(tmem + lane_addr + 384 + cchunk * 32, o);
         tmem_ld_wait();
         if (qrow < S) {
 #pragma unroll
@@ -567,24 +620,23 @@ static_assert(kSmemDkdv <= 232448 && kSmemDq <= 232448, "shared memory");
 static_assert(kSmemDkdv > 232448 / 2 && kSmemDq > 232448 / 2, "one CTA per SM");
 
 template <int HD>
-cudaError_t launch_hd(int BH, int S, float scale, const CUtensorMap* maps_q, const CUtensorMap* maps_kv,
-                      const float* lse, const float* delta, lh_bf16* dqg, lh_bf16* dkg, lh_bf16* dvg,
-                      int* status, cudaStream_t st, int which) {
-  // maps_q: Q, K, V, dO with 64-row boxes (walked tiles of the dK/dV kernel and
-  // K/V of the dQ kernel); maps_kv: the same tensors with 128-row boxes.
+cudaError_t launch_hd(int BH, int S, float scale, const CUtensorMap* maps, const float* lse,
+                      const float* delta, lh_bf16* dqg, lh_bf16* dkg, lh_bf16* dvg, int* status,
+                      cudaStream_t st, int which) {
+  // maps: Q, K, V, dO with 128-row boxes (every tile of both kernels)
   if (which & 1) {
     cudaFuncSetAttribute(k_attn_bwd_dkdv<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemDkdv);
     const int n_kt = (S + KV_M - 1) / KV_M;
     k_attn_bwd_dkdv<HD><<<n_kt * BH, kThreadsDkdv, kSmemDkdv, st>>>(
-        maps_kv[0], maps_kv[1], maps_kv[2], maps_kv[3], lse, delta, (uint4*)dkg, (uint4*)dvg, S, BH,
-        scale, status);
+        maps[0], maps[1], maps[2], maps[3], lse, delta, (uint4*)dkg, (uint4*)dvg, S, BH, scale,
+        status);
   }
   if (which & 2) {
     cudaFuncSetAttribute(k_attn_bwd_dq<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemDq);
     const int n_qt = (S + Q_M - 1) / Q_M;
-    k_attn_bwd_dq<HD><<<n_qt * BH, kThreads, kSmemDq, st>>>(maps_kv[0], maps_q[1], maps_q[2],
-                                                           maps_kv[3], lse, delta, (uint4*)dqg, S,
-                                                           BH, scale, status);
+    k_attn_bwd_dq<HD><<<n_qt * BH, kThreadsDq, kSmemDq, st>>>(maps[0], maps[1], maps[2], maps[3],
+                                                             lse, delta, (uint4*)dqg, S, BH, scale,
+                                                             status);
   }
   return cudaGetLastError();
 }
@@ -599,15 +651,13 @@ cudaError_t lh_launch_attn_bwd(int BH, int64_t S, int d, float scale, const lh_b
                                const float* lse, const float* delta, lh_bf16* dqg,
                                lh_bf16* dkg, lh_bf16* dvg, int* status, cudaStream_t st,
                                int which) {
-  CUtensorMap m64[4], m128[4];
+  CUtensorMap maps[4];
   const lh_bf16* src[4] = {qg, kg, vg, dog};
   for (int i = 0; i < 4; ++i)
-    if (!lh_make_tmap_3d(&m64[i], src[i], BH, S, d, 64) ||
-        !lh_make_tmap_3d(&m128[i], src[i], BH, S, d, 128))
-      return cudaErrorInvalidValue;
+    if (!lh_make_tmap_3d(&maps[i], src[i], BH, S, d, 128)) return cudaErrorInvalidValue;
   if (d == 128)
-    return launch_hd<128>(BH, (int)S, scale, m64, m128, lse, delta, dqg, dkg, dvg, status, st, which);
+    return launch_hd<128>(BH, (int)S, scale, maps, lse, delta, dqg, dkg, dvg, status, st, which);
   if (d == 64)
-    return launch_hd<64>(BH, (int)S, scale, m64, m128, lse, delta, dqg, dkg, dvg, status, st, which);
+    return launch_hd<64>(BH, (int)S, scale, maps, lse, delta, dqg, dkg, dvg, status, st, which);
   return cudaErrorInvalidValue;
 }

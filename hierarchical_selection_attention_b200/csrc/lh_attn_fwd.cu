@@ -4,27 +4,29 @@
 // the mask is the plain S x S causal one, so this is a causal attention
 // forward on [BH, S, d] bf16 tensors, written for the sm_100a tensor cores.
 //
-// One CTA owns two tiles of 128 query rows of one (b, h), A and B (rows
-// 256 g .. 256 g + 255), and walks the key/value tiles of 128 rows up to B's
-// diagonal (A skips the last one).  Warp roles:
-//   warp 0      TMA producer: Q_A and Q_B once, then K and V tiles into a
-//               2-stage ring;
-//   warp 1      tcgen05 issuer (one thread).  Per key tile j it issues
-//               S_A = Q_A K^T, S_B = Q_B K^T into TMEM, then, as each softmax
-//               warpgroup hands back its P, O_X += P_X V with P_X read from
-//               TMEM (A operand in tensor memory) and V from shared memory;
-//   warps 2-5   softmax of tile A, warps 6-9 softmax of tile B: one query
-//               row per thread (TMEM lane = row).  Each reads its score row,
-//               keeps the exact running max and the row sum, writes
-//               P = exp2(s - max) as bf16 pairs over the score columns it
-//               has just read, and rescales O_X in TMEM when a row's max grew.
-// While warpgroup A turns S_A into P_A, the tensor core works on S_B or on
-// P_B V, and the other way round.
+// One CTA owns one tile of 128 query rows of one (b, h) and walks the
+// key/value tiles of 128 rows up to its diagonal.  Warp roles:
+//   warp 0      TMA producer: Q once, then K and V tiles into their rings;
+//   warp 1      issuer A: S(j) = Q K(j)^T into TMEM score buffer j % 2;
+//   warp 10     issuer B: O_h += P_h(j) V_h(j) for the two column halves h
+//               (keys 64 h .. 64 h + 63 of the tile), P_h read from TMEM (A
+//               operand in tensor memory), V from shared memory;
+//   warps 2-9   two softmax warpgroups; warpgroup h owns columns 64 h ..
+//               64 h + 63 of every score row, one row per thread (TMEM lane
+//               = row), with its own exact running max, row sum and output
+//               accumulator O_h: a split of the key dimension in two inside
+//               the CTA, so the warpgroups never exchange anything per tile.
+//               The epilogue merges the halves: with m = max(m_0, m_1),
+//               O = (O_0 2^(m_0 - m) + O_1 2^(m_1 - m)) / (l_0 2^(m_0 - m) +
+//               l_1 2^(m_1 - m)).
+// With two score buffers S(j + 1) is computed while the softmax works on
+// S(j), and P(j) V(j) runs while it works on S(j + 1), so the tensor pipe and
+// the softmax overlap.  The issuers run whole-warp loops (one lane issues).
 //
-// TMEM (512 columns, one CTA per SM): S_A 0..127, S_B 128..255 (P_X packed
-// into the first 64 columns of S_X), O_A and O_B (d columns each) from 256.
-// Shared memory: Q_A, Q_B, two K and two V stages (128 x d bf16 each),
-// 128-byte swizzled, 1024-byte aligned.
+// TMEM (512 columns, one CTA per SM): score buffers 0..127 and 128..255
+// (P_h packed into the first 32 columns of its half), O_0 from 256 and O_1
+// from 256 + d.  Shared memory: Q, KST K stages and VST V stages (128 x d
+// bf16 each), 128-byte swizzled, 1024-byte aligned, and the merge buffer.
 #include <cudaTypedefs.h>
 
 #include "lh_sm100.cuh"
@@ -35,16 +37,19 @@ using namespace sm100;
 
 constexpr int BM = 128;
 constexpr int BN = 128;
-constexpr int NST = 2;
-constexpr int kThreads = 320;
+constexpr int KST = 3;
+constexpr int VST = 2;
+constexpr int kThreads = 352;
+constexpr int kHalf = 128;           // threads of one softmax warpgroup
 constexpr uint32_t kTmemCols = 512;
 
 template <int HD>
 struct FwdLayout {
-  static constexpr uint32_t q = 0;                       // Q_A, Q_B
-  static constexpr uint32_t k = q + 2 * BM * HD * 2;
-  static constexpr uint32_t v = k + NST * BN * HD * 2;
-  static constexpr uint32_t bar = v + NST * BN * HD * 2;
+  static constexpr uint32_t q = 0;
+  static constexpr uint32_t k = q + BM * HD * 2;
+  static constexpr uint32_t v = k + KST * BN * HD * 2;
+  static constexpr uint32_t merge = v + VST * BN * HD * 2;   // [2][128] (m, l) pairs
+  static constexpr uint32_t bar = merge + 2 * BM * 8;
   static constexpr uint32_t bytes = bar + 256;
 };
 
@@ -54,9 +59,11 @@ constexpr uint32_t kSmemBytes = FwdLayout<128>::bytes + 1024;
 static_assert(kSmemBytes > 232448 / 2 && kSmemBytes <= 232448, "one CTA per SM");
 
 struct Bars {
+  // Indexed by score buffer (tile parity), so a fast side can never
+  // complete a barrier twice before the other side has seen the first phase.
   uint64_t qfull;
-  uint64_t kfull[NST], kempty[NST], vfull[NST], vempty[NST];
-  uint64_t sfull[2], pfull[2], odone[2];
+  uint64_t kfull[KST], kempty[KST], vfull[VST], vempty[VST];
+  uint64_t sfull[2], pfull[2][2], pvdone[2];
   uint32_t tmem_base;
 };
 
@@ -71,33 +78,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
   Bars* bars = reinterpret_cast<Bars*>(smem + Lay::bar);
-  const uint32_t sQ = smem_u32(smem + Lay::q);
-  const uint32_t sK = smem_u32(smem + Lay::k);
-  const uint32_t sV = smem_u32(smem + Lay::v);
-
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n_qt = (S + BM - 1) / BM;
-  const int n_pair = (n_qt + 1) / 2;
-  const int g = n_pair - 1 - (int)(blockIdx.x / BH);  // longest rows first
+  const int qt = n_qt - 1 - (int)(blockIdx.x / BH);  // longest rows first
   const int bh = (int)(blockIdx.x % BH);
-  const int qt_a = 2 * g, qt_b = 2 * g + 1;
-  const int n_a = qt_a + 1;                           // key tiles of tile A
-  const int n_b = qt_b < n_qt ? qt_b + 1 : 0;         // 0: tile B is past the end
-  const int n_kv = n_b ? n_b : n_a;
+  const int n_kv = qt + 1;                           // key tiles up to the diagonal (BN == BM)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->qfull, 1);
-    for (int s = 0; s < NST; ++s) {
+    for (int s = 0; s < KST; ++s) {
       mbar_init(&bars->kfull[s], 1);
       mbar_init(&bars->kempty[s], 1);
+    }
+    for (int s = 0; s < VST; ++s) {
       mbar_init(&bars->vfull[s], 1);
       mbar_init(&bars->vempty[s], 1);
     }
-    for (int x = 0; x < 2; ++x) {
-      mbar_init(&bars->sfull[x], 1);
-      mbar_init(&bars->pfull[x], 128);
-      mbar_init(&bars->odone[x], 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->sfull[b], 1);
+      mbar_init(&bars->pfull[b][0], kHalf);
+      mbar_init(&bars->pfull[b][1], kHalf);
+      mbar_init(&bars->pvdone[b], 1);
     }
     fence_mbar_init();
   }
@@ -115,157 +117,141 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_expect_tx(&bars->qfull, 2 * BM * HD * 2);
-      for (int x = 0; x < 2; ++x)
-        for (int blk = 0; blk < HD / 64; ++blk)
-          tma_load_3d(&tmQ, &bars->qfull, smem + Lay::q + x * BM * HD * 2 + blk * BM * 128,
-                      64 * blk, (qt_a + x) * BM, bh);
+      mbar_expect_tx(&bars->qfull, BM * HD * 2);
+      for (int blk = 0; blk < HD / 64; ++blk)
+        tma_load_3d(&tmQ, &bars->qfull, smem + Lay::q + blk * BM * 128, 64 * blk, qt * BM, bh);
       for (int j = 0; j < n_kv; ++j) {
-        const int s = j % NST;
-        const uint32_t ph = (j / NST) & 1;
-        if (!mbar_wait(&bars->kempty[s], ph ^ 1, status, 1)) break;
+        const int s = j % KST, t = j % VST;
+        if (!mbar_wait(&bars->kempty[s], ((j / KST) & 1) ^ 1, status, 1)) break;
         mbar_expect_tx(&bars->kfull[s], BN * HD * 2);
         for (int blk = 0; blk < HD / 64; ++blk)
           tma_load_3d(&tmK, &bars->kfull[s], smem + Lay::k + s * BN * HD * 2 + blk * BN * 128,
                       64 * blk, j * BN, bh);
-        if (!mbar_wait(&bars->vempty[s], ph ^ 1, status, 2)) break;
-        mbar_expect_tx(&bars->vfull[s], BN * HD * 2);
+        if (!mbar_wait(&bars->vempty[t], ((j / VST) & 1) ^ 1, status, 2)) break;
+        mbar_expect_tx(&bars->vfull[t], BN * HD * 2);
         for (int blk = 0; blk < HD / 64; ++blk)
-          tma_load_3d(&tmV, &bars->vfull[s], smem + Lay::v + s * BN * HD * 2 + blk * BN * 128,
+          tma_load_3d(&tmV, &bars->vfull[t], smem + Lay::v + t * BN * HD * 2 + blk * BN * 128,
                       64 * blk, j * BN, bh);
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16(BM, BN, 0, 0);
-      constexpr uint32_t idO = idesc_bf16(BM, HD, 0, 1);
-      bool ok = mbar_wait(&bars->qfull, 0, status, 3);
-      for (int j = 0; ok && j < n_kv; ++j) {
-        const int s = j % NST;
-        const uint32_t ph = (j / NST) & 1;
-        if (!mbar_wait(&bars->kfull[s], ph, status, 4)) { ok = false; break; }
-        const uint32_t kb = sK + s * BN * HD * 2;
-        for (int x = 0; x < 2 && ok; ++x) {
-          if (j >= (x ? n_b : n_a)) continue;
-          // S_X shares its columns with P_X of the last tile: P_X V must be done
-          if (j > 0 && !mbar_wait(&bars->odone[x], (j - 1) & 1, status, 5)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t qb = sQ + x * BM * HD * 2;
+    // Issuer A: S(j) = Q K(j)^T into buffer j % 2, once P(j - 2) V(j - 2)
+    // (which read P(j - 2) from that buffer) has finished.
+    constexpr uint32_t idS = idesc_bf16(BM, BN, 0, 0);
+    const uint32_t sQ = smem_u32(smem + Lay::q), sK = smem_u32(smem + Lay::k);
+    bool ok = mbar_wait_w(&bars->qfull, 0, status, 3);
+    for (int j = 0; ok && j < n_kv; ++j) {
+      const int s = j % KST, b = j & 1;
+      if (!mbar_wait_w(&bars->kfull[s], (j / KST) & 1, status, 4)) break;
+      if (j >= 2 && !mbar_wait_w(&bars->pvdone[b], ((j >> 1) & 1) ^ 1, status, 5)) break;
+      tc_fence_after();
+      const uint32_t kb = sK + s * BN * HD * 2;
 #pragma unroll
-          for (int ks = 0; ks < HD / 16; ++ks) {
-            const uint64_t a = sdesc_sw128(qb + (ks >> 2) * BM * 128 + (ks & 3) * 32, 16, 1024);
-            const uint64_t b = sdesc_sw128(kb + (ks >> 2) * BN * 128 + (ks & 3) * 32, 16, 1024);
-            mma_bf16(tmem + x * 128, a, b, idS, ks > 0 ? 1u : 0u);
-          }
-          mma_commit(&bars->sfull[x]);
-        }
-        if (!ok) break;
-        mma_commit(&bars->kempty[s]);
-        if (!mbar_wait(&bars->vfull[s], ph, status, 6)) { ok = false; break; }
-        const uint32_t vb = sV + s * BN * HD * 2;
-        for (int x = 0; x < 2 && ok; ++x) {
-          if (j >= (x ? n_b : n_a)) continue;
-          if (!mbar_wait(&bars->pfull[x], j & 1, status, 7)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int ks = 0; ks < BN / 16; ++ks) {
-            const uint64_t b = sdesc_sw128(vb + ks * 16 * 128, BN * 128, 1024);
-            mma_bf16_ts(tmem + 256 + x * HD, tmem + x * 128 + ks * 8, b, idO,
-                        (j > 0 || ks > 0) ? 1u : 0u);
-          }
-          mma_commit(&bars->odone[x]);
-        }
-        if (!ok) break;
-        mma_commit(&bars->vempty[s]);
+      for (int ks = 0; ks < HD / 16; ++ks) {
+        const uint64_t a = sdesc_sw128(sQ + (ks >> 2) * BM * 128 + (ks & 3) * 32, 16, 1024);
+        const uint64_t bd = sdesc_sw128(kb + (ks >> 2) * BN * 128 + (ks & 3) * 32, 16, 1024);
+        mma_bf16_w(tmem + b * BN, a, bd, idS, ks > 0 ? 1u : 0u);
       }
+      mma_commit_w(&bars->sfull[b]);
+      mma_commit_w(&bars->kempty[s]);
+    }
+  } else if (warp == 10) {
+    // Issuer B: O_h += P_h(j) V_h(j) as each softmax warpgroup hands back its
+    // half of P(j) (and has rescaled O_h for tile j's max).
+    constexpr uint32_t idO = idesc_bf16(BM, HD, 0, 1);
+    const uint32_t sV = smem_u32(smem + Lay::v);
+    bool ok = true;
+    for (int j = 0; ok && j < n_kv; ++j) {
+      const int t = j % VST, b = j & 1;
+      if (!mbar_wait_w(&bars->vfull[t], (j / VST) & 1, status, 6)) break;
+      const uint32_t vb = sV + t * BN * HD * 2;
+      for (int h = 0; h < 2; ++h) {
+        if (!mbar_wait_w(&bars->pfull[b][h], (j >> 1) & 1, status, 7)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < BN / 32; ++ks)
+          mma_bf16_ts_w(tmem + 256 + h * HD, tmem + b * BN + h * 64 + ks * 8,
+                        sdesc_sw128(vb + (h * 4 + ks) * 16 * 128, BN * 128, 1024), idO,
+                        (j > 0 || ks > 0) ? 1u : 0u);
+      }
+      if (!ok) break;
+      mma_commit_w(&bars->pvdone[b]);
+      mma_commit_w(&bars->vempty[t]);
     }
   } else {
-    // softmax warpgroup x: warps 2-5 (x = 0) and 6-9 (x = 1)
-    const int x = (warp - 2) >> 2;
+    // softmax warpgroup h (warps 2-5: h = 0, 6-9: h = 1); TMEM lane quarter =
+    // warp % 4.  Waits are warp-wide (the vote below needs every lane).
+    const int h = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;       // row in the tile = TMEM lane
-    const int qt = qt_a + x;
     const int qrow = qt * BM + r;            // row in the sequence
-    const int n_x = x ? n_b : n_a;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_addr + x * 128;
-    const uint32_t tO = tmem + lane_addr + 256 + x * HD;
+    const uint32_t tO = tmem + lane_addr + 256 + h * HD;
+    const int c0 = h * 64;                   // first column of this half
     float m_used = -INFINITY, lsum = 0.f;
     bool ok = true;
-    for (int j = 0; j < n_x; ++j) {
-      if (!mbar_wait(&bars->sfull[x], j & 1, status, 8)) { ok = false; break; }
+    for (int j = 0; j < n_kv; ++j) {
+      const int b = j & 1;
+      const uint32_t tS = tmem + lane_addr + b * BN + c0;
+      if (!mbar_wait_w(&bars->sfull[b], (j >> 1) & 1, status, 8)) { ok = false; break; }
       tc_fence_after();
-      // Two passes over the score row in TMEM, two 32-column chunks at a
-      // time: the max first, then exp2 / sum / pack.  Holding the whole row
-      // in registers would spill at this block size.
+      uint32_t s[64];
+      tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+      tmem_ld_wait();
       const bool diag = (j == qt);
       float mxv[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) mxv[u] = -INFINITY;
+      if (diag) {
 #pragma unroll
-      for (int c = 0; c < BN / 32; c += 2) {
-        uint32_t a[32], b[32];
-        tmem_ld32(tS + c * 32, a);
-        tmem_ld32(tS + c * 32 + 32, b);
-        tmem_ld_wait();
-        if (diag) {
+        for (int e = 0; e < 64; ++e)
+          if (c0 + e <= r) mxv[e & 7] = fmaxf(mxv[e & 7], __uint_as_float(s[e]));
+      } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            if (c * 32 + e <= r) mxv[e & 7] = fmaxf(mxv[e & 7], __uint_as_float(a[e]));
-            if (c * 32 + 32 + e <= r) mxv[e & 7] = fmaxf(mxv[e & 7], __uint_as_float(b[e]));
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            mxv[e & 7] = fmaxf(mxv[e & 7], fmaxf(__uint_as_float(a[e]), __uint_as_float(b[e])));
-        }
+        for (int e = 0; e < 64; ++e) mxv[e & 7] = fmaxf(mxv[e & 7], __uint_as_float(s[e]));
       }
       const float mx = fmaxf(fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3])),
                              fmaxf(fmaxf(mxv[4], mxv[5]), fmaxf(mxv[6], mxv[7])));
-      // Exact running max: the row's largest term so far gets p = 1, which
-      // bf16 holds exactly.  (A stale max, as lazy rescaling keeps, would
-      // round that dominant term by up to 2^-9, and the error would reach
-      // D = rowsum(dO * O) of the backward unscaled.)
+      // Exact running max (of this half): the largest term so far gets
+      // p = 1, which bf16 holds exactly.  (A stale max, as lazy rescaling
+      // keeps, would round that dominant term by up to 2^-9, and the error
+      // would reach D = rowsum(dO * O) of the backward unscaled.)  A half
+      // whose columns are all masked so far keeps m = -inf and p = 0.
       const float m_new = fmaxf(m_used, mx * scale_log2);
       const bool grow = m_new > m_used;
       const float alpha = grow ? ex2(m_used - m_new) : 1.f;
       m_used = m_new;
+      const float m_sub = m_used == -INFINITY ? 0.f : m_used;
       float rsv[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) rsv[u] = 0.f;
 #pragma unroll
-      for (int c = 0; c < BN / 32; c += 2) {
-        uint32_t a[32], b[32];
-        tmem_ld32(tS + c * 32, a);
-        tmem_ld32(tS + c * 32 + 32, b);
-        tmem_ld_wait();
-        uint32_t pa[16], pb[16];
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[8];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float p0 = ex2(fmaf(__uint_as_float(a[e]), scale_log2, -m_used));
-          float p1 = ex2(fmaf(__uint_as_float(a[e + 1]), scale_log2, -m_used));
-          float q0 = ex2(fmaf(__uint_as_float(b[e]), scale_log2, -m_used));
-          float q1 = ex2(fmaf(__uint_as_float(b[e + 1]), scale_log2, -m_used));
+        for (int e = 0; e < 16; e += 2) {
+          const int i = c * 16 + e;
+          float p0 = ex2(fmaf(__uint_as_float(s[i]), scale_log2, -m_sub));
+          float p1 = ex2(fmaf(__uint_as_float(s[i + 1]), scale_log2, -m_sub));
           if (diag) {
-            p0 = (c * 32 + e <= r) ? p0 : 0.f;
-            p1 = (c * 32 + e + 1 <= r) ? p1 : 0.f;
-            q0 = (c * 32 + 32 + e <= r) ? q0 : 0.f;
-            q1 = (c * 32 + 32 + e + 1 <= r) ? q1 : 0.f;
+            p0 = (c0 + i <= r) ? p0 : 0.f;
+            p1 = (c0 + i + 1 <= r) ? p1 : 0.f;
           }
-          rsv[(e >> 1) & 7] += (p0 + p1) + (q0 + q1);
-          pa[e >> 1] = pack_bf16x2(p0, p1);
-          pb[e >> 1] = pack_bf16x2(q0, q1);
+          rsv[(i >> 1) & 7] += p0 + p1;
+          pk[e >> 1] = pack_bf16x2(p0, p1);
         }
-        // P over columns of this row already read (pair c covers 64 score
-        // columns from c * 32 and packs into 32 columns from c * 16)
-        tmem_st16(tS + c * 16, pa);
-        tmem_st16(tS + c * 16 + 16, pb);
+        // P of columns 16 c .. 16 c + 15 of this half lands on columns
+        // 8 c .. 8 c + 7, whose scores were read above
+        tmem_st8(tS + c * 8, pk);
       }
       const float rs = ((rsv[0] + rsv[1]) + (rsv[2] + rsv[3])) + ((rsv[4] + rsv[5]) + (rsv[6] + rsv[7]));
       lsum = lsum * alpha + rs;
-      // O_X holds P V of the earlier tiles (P_X V of tile j-1 finished before
-      // S_X of tile j was issued); bring it to the new max.
+      // O_h holds P_h V_h of the earlier tiles; bring it to the new max once
+      // P(j - 1) V(j - 1) has finished.
       if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        if (!mbar_wait_w(&bars->pvdone[(j - 1) & 1], ((j - 1) >> 1) & 1, status, 9)) { ok = false; break; }
+        tc_fence_after();
 #pragma unroll
         for (int c = 0; c < HD / 32; ++c) {
           uint32_t o[32];
@@ -278,15 +264,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bars->pfull[x]);
+      mbar_arrive(&bars->pfull[b][h]);
     }
-    if (ok && n_x > 0 && mbar_wait(&bars->odone[x], (n_x - 1) & 1, status, 10)) {
+    // ---- merge the two halves; warpgroup h writes output columns
+    // HD/2 h .. HD/2 h + HD/2 - 1
+    float2* mg = reinterpret_cast<float2*>(smem + Lay::merge);
+    mg[h * BM + r] = make_float2(m_used, lsum);
+    named_bar(1, 2 * kHalf);
+    const float2 o_ml = mg[(h ^ 1) * BM + r];
+    if (ok && mbar_wait_w(&bars->pvdone[(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, status, 10)) {
       tc_fence_after();
-      const float inv = 1.f / lsum;
+      const float m0 = h ? o_ml.x : m_used, l0 = h ? o_ml.y : lsum;
+      const float m1 = h ? m_used : o_ml.x, l1 = h ? lsum : o_ml.y;
+      const float m = fmaxf(m0, m1);                 // finite: column 0 is never masked
+      const float a0 = ex2(m0 - m), a1 = ex2(m1 - m);
+      const float l = l0 * a0 + l1 * a1;
+      const float inv = 1.f / l;
+      const float w0 = a0 * inv, w1 = a1 * inv;
+      const uint32_t tO0 = tmem + lane_addr + 256, tO1 = tO0 + HD;
 #pragma unroll
-      for (int c = 0; c < HD / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tO + c * 32, o);
+      for (int cc = 0; cc < HD / 64; ++cc) {
+        const int c = h * (HD / 64) + cc;            // 32-column chunk of the output
+        uint32_t o0[32], o1[32];
+        tmem_ld32(tO0 + c * 32, o0);
+        tmem_ld32(tO1 + c * 32, o1);
         tmem_ld_wait();
         if (qrow < S) {
           const int64_t base = ((int64_t)bh * S + qrow) * (HD / 8) + c * 4;
@@ -294,7 +295,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int v = 0; v < 4; ++v) {
             float xv[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) xv[e] = __uint_as_float(o[v * 8 + e]) * inv;
+            for (int e = 0; e < 8; ++e)
+              xv[e] = __uint_as_float(o0[v * 8 + e]) * w0 + __uint_as_float(o1[v * 8 + e]) * w1;
             uint4 w;
             w.x = pack_bf16x2(xv[0], xv[1]); w.y = pack_bf16x2(xv[2], xv[3]);
             w.z = pack_bf16x2(xv[4], xv[5]); w.w = pack_bf16x2(xv[6], xv[7]);
@@ -312,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (qrow < S) lse[(int64_t)bh * S + qrow] = (m_used + __log2f(lsum)) * 0.69314718055994531f;
+      if (h == 0 && qrow < S) lse[(int64_t)bh * S + qrow] = (m + __log2f(l)) * 0.69314718055994531f;
     }
     tc_fence_before();
   }
@@ -362,7 +364,7 @@ cudaError_t lh_launch_attn_fwd(int BH, int64_t S, int d, float scale, const lh_b
       !lh_make_tmap_3d(&tv, vg, BH, S, d, BN))
     return cudaErrorInvalidValue;
   const int n_qt = (int)((S + BM - 1) / BM);
-  const dim3 grid((unsigned)(((n_qt + 1) / 2) * BH));
+  const dim3 grid((unsigned)(n_qt * BH));
   const float scale_log2 = scale * 1.4426950408889634f;
   if (d == 128) {
     cudaFuncSetAttribute(k_attn_fwd<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);

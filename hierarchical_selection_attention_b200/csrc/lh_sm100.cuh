@@ -294,6 +294,15 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Forces the 16 values to be computed here: the empty volatile asm cannot
+// move across the barrier waits around it, so the arithmetic feeding it
+// (e.g. exponentials) is not sunk past a wait it could overlap.
+__device__ __forceinline__ void materialize16(const uint32_t* r) {
+  asm volatile("" ::"r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+               "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]),
+               "r"(r[14]), "r"(r[15]));
+}
+
 // 2^x evaluated on the FMA pipe instead of the special-function unit, for
 // kernels whose exponentials saturate that unit (16 per clock per SM): the
 // caller sends a fraction of its elements here.  x = n + f with n the
