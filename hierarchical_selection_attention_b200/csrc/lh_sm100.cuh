@@ -303,25 +303,6 @@ __device__ __forceinline__ void materialize16(const uint32_t* r) {
                "r"(r[14]), "r"(r[15]));
 }
 
-// 2^x evaluated on the FMA pipe instead of the special-function unit, for
-// kernels whose exponentials saturate that unit (16 per clock per SM): the
-// caller sends a fraction of its elements here.  x = n + f with n the
-// nearest integer (rounded by adding 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f
-// by a degree-4 polynomial that interpolates 2^f at the five Chebyshev nodes
-// of [-1/2, 1/2] (coefficients from fit_exp2_poly.py beside this file,
-// maximum relative error 3.6e-6); 2^n is added into the exponent field.
-// Valid for -126 <= x < 128; smaller x is clamped to -126.
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -126.f);
-  const float t = x + 12582912.f;
-  const float f = x - (t - 12582912.f);
-  float p = fmaf(0x1.3cbf60p-7f, f, 0x1.ca1ce2p-5f);
-  p = fmaf(p, f, 0x1.ebfa4cp-3f);
-  p = fmaf(p, f, 0x1.62e0c2p-1f);
-  p = fmaf(p, f, 1.0f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 // Named barrier over `nthreads` threads (multiple of 32) with id `id` (1..15).
 __device__ __forceinline__ void named_bar(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
