@@ -267,6 +267,7 @@ __global__ void __launch_bounds__(kThreadsDkdv, 1)
       const bool diag = it == 0;
       // ---- P = exp2(c (s - LSE / scale)): fp32 kept in registers, bf16 into TMEM
       uint32_t p[64];                                // scores, then P (fp32 bits)
+      const uint64_t c2 = f2_pack(c, c);
       if (!mbar_wait(&bars->sfull, it & 1, status, 27)) { ok = false; break; }
       tc_fence_after();
       tmem_ld32(cS, *reinterpret_cast<uint32_t(*)[32]>(&p[0]));
@@ -278,9 +279,9 @@ __global__ void __launch_bounds__(kThreadsDkdv, 1)
 #pragma unroll
         for (int e = 0; e < 16; e += 2) {
           const int j = ch * 16 + e;
-          const float x0 = __uint_as_float(p[j]) * c, x1 = __uint_as_float(p[j + 1]) * c;
-          float p0 = ex2(x0);
-          float p1 = ex2(x1);
+          const float2 x = f2_unpack(f2_mul(f2_pack(__uint_as_float(p[j]), __uint_as_float(p[j + 1])), c2));
+          float p0 = ex2(x.x);
+          float p1 = ex2(x.y);
           if (diag) {
             p0 = (qc0 + j >= kvrow) ? p0 : 0.f;
             p1 = (qc0 + j + 1 >= kvrow) ? p1 : 0.f;
@@ -310,8 +311,9 @@ __global__ void __launch_bounds__(kThreadsDkdv, 1)
 #pragma unroll
         for (int e = 0; e < 16; e += 2) {
           const int j = ch * 16 + e;
-          dk[e >> 1] = pack_bf16x2(__uint_as_float(p[j]) * __uint_as_float(q[e]),
-                                   __uint_as_float(p[j + 1]) * __uint_as_float(q[e + 1]));
+          const float2 ds = f2_unpack(f2_mul(f2_pack(__uint_as_float(p[j]), __uint_as_float(p[j + 1])),
+                                             f2_pack(__uint_as_float(q[e]), __uint_as_float(q[e + 1]))));
+          dk[e >> 1] = pack_bf16x2(ds.x, ds.y);
         }
         // chunk ch's packed dS covers fp32 columns 8 ch .. 8 ch + 7, all
         // read by the loads of chunks <= ch, which have completed
@@ -548,17 +550,24 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&bars->sfree[sb]);
+      const uint64_t c2 = f2_pack(c, c), nl2 = f2_pack(-lrow, -lrow);
 #pragma unroll
-      for (int e = 0; e < 64; ++e) {
-        float pv = ex2(fmaf(__uint_as_float(p[e]), c, -lrow));
-        if (diag) pv = (kc0 + e <= qrow) ? pv : 0.f;
-        p[e] = __float_as_uint(pv);
+      for (int e = 0; e < 64; e += 2) {
+        const float2 x = f2_unpack(f2_fma(f2_pack(__uint_as_float(p[e]), __uint_as_float(p[e + 1])), c2, nl2));
+        float p0 = ex2(x.x), p1 = ex2(x.y);
+        if (diag) {
+          p0 = (kc0 + e <= qrow) ? p0 : 0.f;
+          p1 = (kc0 + e + 1 <= qrow) ? p1 : 0.f;
+        }
+        p[e] = __float_as_uint(p0);
+        p[e + 1] = __float_as_uint(p1);
       }
 #pragma unroll
       for (int g = 0; g < 4; ++g) materialize16(p + 16 * g);
       // ---- dS = P (dP - D), bf16 into TMEM; the dP loads run one chunk ahead
       if (!mbar_wait(&bars->dpfull, j & 1, status, 39)) { ok = false; break; }
       tc_fence_after();
+      const uint64_t nd2 = f2_pack(-drow, -drow);
       uint32_t pr[2][16];
       tmem_ld16(cP, pr[0]);
       tmem_ld_wait();
@@ -570,8 +579,9 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
 #pragma unroll
         for (int e = 0; e < 16; e += 2) {
           const int i = ch * 16 + e;
-          dk[e >> 1] = pack_bf16x2(__uint_as_float(p[i]) * (__uint_as_float(q[e]) - drow),
-                                   __uint_as_float(p[i + 1]) * (__uint_as_float(q[e + 1]) - drow));
+          const float2 ds = f2_unpack(f2_mul(f2_pack(__uint_as_float(p[i]), __uint_as_float(p[i + 1])),
+                                             f2_add(f2_pack(__uint_as_float(q[e]), __uint_as_float(q[e + 1])), nd2)));
+          dk[e >> 1] = pack_bf16x2(ds.x, ds.y);
         }
         // chunk ch's packed dS covers fp32 columns 8 ch .. 8 ch + 7, all
         // read by the loads of chunks <= ch, which have completed

@@ -209,7 +209,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (c0 + e <= r) mxv[e & 7] = fmaxf(mxv[e & 7], __uint_as_float(s[e]));
       } else {
 #pragma unroll
-        for (int e = 0; e < 64; ++e) mxv[e & 7] = fmaxf(mxv[e & 7], __uint_as_float(s[e]));
+        for (int e = 0; e < 64; e += 2)
+          mxv[(e >> 1) & 7] = fmax3(mxv[(e >> 1) & 7], __uint_as_float(s[e]), __uint_as_float(s[e + 1]));
       }
       const float mx = fmaxf(fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3])),
                              fmaxf(fmaxf(mxv[4], mxv[5]), fmaxf(mxv[6], mxv[7])));
@@ -223,29 +224,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float alpha = grow ? ex2(m_used - m_new) : 1.f;
       m_used = m_new;
       const float m_sub = m_used == -INFINITY ? 0.f : m_used;
-      float rsv[8];
+      // x = s scale - m and the row sum in packed fp32 pairs
+      const uint64_t sc2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(-m_sub, -m_sub);
+      uint64_t rs2[4];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) rsv[u] = 0.f;
+      for (int u = 0; u < 4; ++u) rs2[u] = f2_pack(0.f, 0.f);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[8];
 #pragma unroll
         for (int e = 0; e < 16; e += 2) {
           const int i = c * 16 + e;
-          float p0 = ex2(fmaf(__uint_as_float(s[i]), scale_log2, -m_sub));
-          float p1 = ex2(fmaf(__uint_as_float(s[i + 1]), scale_log2, -m_sub));
+          const float2 x = f2_unpack(f2_fma(f2_pack(__uint_as_float(s[i]), __uint_as_float(s[i + 1])), sc2, nm2));
+          float p0 = ex2(x.x), p1 = ex2(x.y);
           if (diag) {
             p0 = (c0 + i <= r) ? p0 : 0.f;
             p1 = (c0 + i + 1 <= r) ? p1 : 0.f;
           }
-          rsv[(i >> 1) & 7] += p0 + p1;
+          rs2[(i >> 1) & 3] = f2_add(rs2[(i >> 1) & 3], f2_pack(p0, p1));
           pk[e >> 1] = pack_bf16x2(p0, p1);
         }
         // P of columns 16 c .. 16 c + 15 of this half lands on columns
         // 8 c .. 8 c + 7, whose scores were read above
         tmem_st8(tS + c * 8, pk);
       }
-      const float rs = ((rsv[0] + rsv[1]) + (rsv[2] + rsv[3])) + ((rsv[4] + rsv[5]) + (rsv[6] + rsv[7]));
+      const float2 ra = f2_unpack(f2_add(rs2[0], rs2[1])), rb = f2_unpack(f2_add(rs2[2], rs2[3]));
+      const float rs = (ra.x + ra.y) + (rb.x + rb.y);
       lsum = lsum * alpha + rs;
       // O_h holds P_h V_h of the earlier tiles; bring it to the new max once
       // P(j - 1) V(j - 1) has finished.
