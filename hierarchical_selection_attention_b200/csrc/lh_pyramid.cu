@@ -112,13 +112,18 @@ __global__ void __launch_bounds__(256, 2) k_pyramid_score(LhDims D, const uint4*
         const int64_t i = ent[l]++;
         left[l] = (int)D.lvl_span[l];
         const float fs = (float)D.lvl_span[l];
+        // x / p^l; for a power-of-two span the product with the exact
+        // reciprocal is the same correctly rounded quotient
+        const bool pow2 = (D.lvl_span[l] & (D.lvl_span[l] - 1)) == 0;
+        const float inv = 1.f / fs;
+        auto mean = [&](float x) { return pow2 ? x * inv : __fdiv_rn(x, fs); };
         uint4 oq, ok, ov;
         uint32_t* pq = &oq.x; uint32_t* pk = &ok.x; uint32_t* pv = &ov.x;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          pq[e] = pack_bf16x2(__fdiv_rn(aq[l - 1][2 * e], fs), __fdiv_rn(aq[l - 1][2 * e + 1], fs));
-          pk[e] = pack_bf16x2(__fdiv_rn(ak[l - 1][2 * e], fs), __fdiv_rn(ak[l - 1][2 * e + 1], fs));
-          pv[e] = pack_bf16x2(__fdiv_rn(av[l - 1][2 * e], fs), __fdiv_rn(av[l - 1][2 * e + 1], fs));
+          pq[e] = pack_bf16x2(mean(aq[l - 1][2 * e]), mean(aq[l - 1][2 * e + 1]));
+          pk[e] = pack_bf16x2(mean(ak[l - 1][2 * e]), mean(ak[l - 1][2 * e + 1]));
+          pv[e] = pack_bf16x2(mean(av[l - 1][2 * e]), mean(av[l - 1][2 * e + 1]));
         }
         const int64_t orow = ((int64_t)D.B * D.pool_row[l] + (int64_t)b * D.lvl_size[l] + i) * HV + j;
         q_lv[orow] = oq;
