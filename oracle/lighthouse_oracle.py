@@ -91,13 +91,15 @@ def subseq_len(N: int, L: int, p: int, k: int) -> int:
     return N // p ** (L - 1) + n_select(L, p, k)
 
 
-def check_config(N: int, L: int, p: int, k: int) -> None:
+def check_config(N: int, L: int, p: int, k: int, mode: int = 0) -> None:
     if p < 2 or L < 1 or N < 1 or k < 0:
         raise ValueError("need p >= 2, L >= 1, N >= 1, k >= 0")
     if N % p ** (L - 1):
         raise ValueError("p^(L-1) must divide N (Sec. 3.3)")
     if n_select(L, p, k) > n_candidates(N, L, p):
         raise ValueError("(L-1) p k exceeds the number of finer-level entries")
+    if mode == 1 and L > 1 and p * k > N // p ** (L - 2):
+        raise ValueError("per-level quota: p k exceeds the entries of the coarsest finer level")
 
 
 def entry_level_index(f: np.ndarray, N: int, L: int, p: int):
@@ -177,23 +179,36 @@ def scores(qh: np.ndarray, kh: np.ndarray, L: int, p: int):
     return np.concatenate(qk), np.concatenate(kq)
 
 
-def select(qk: np.ndarray, kq: np.ndarray, N: int, L: int, p: int, k: int) -> np.ndarray:
+def select(qk: np.ndarray, kq: np.ndarray, N: int, L: int, p: int, k: int,
+           mode: int = 0) -> np.ndarray:
     """Selection flags over all flat pyramid indices of one head.
 
-    The QK and KQ streams of the finer levels are concatenated and sorted by
-    score (descending), ties by lower flat index; distinct entries are taken
-    from the front until n_sel are found.  Level L-1 is kept whole.
+    mode 0 (joint, Sec. 3.4): the QK and KQ streams of the finer levels are
+    concatenated and sorted by score (descending), ties by lower flat index;
+    distinct entries are taken from the front until n_sel are found.
+
+    mode 1 (per-level quota, the Eq. 8 accounting read literally: each of
+    the L-1 finer levels contributes p k entries): the same walk, but over
+    one finer level at a time, taking p k distinct entries from each.
+
+    Level L-1 is kept whole in both modes.
     """
     C = n_candidates(N, L, p)
-    n_sel = n_select(L, p, k)
-    f = np.arange(C, dtype=np.int64)
-    stream_f = np.concatenate([f, f])
-    stream_s = np.concatenate([qk[:C], kq[:C]]).astype(np.float64)
-    walk = stream_f[np.lexsort((stream_f, -stream_s))]
-    _, first = np.unique(walk, return_index=True)   # where each entry first shows up
-    chosen = walk[np.sort(first)[:n_sel]]
     flags = np.zeros(total_entries(N, L, p), dtype=bool)
-    flags[chosen] = True
+    if mode == 0:
+        ranges = [(0, C, n_select(L, p, k))]
+    elif mode == 1:
+        offs = level_offsets(N, L, p)
+        ranges = [(offs[l], offs[l] + N // p**l, p * k) for l in range(L - 1)]
+    else:
+        raise ValueError("select mode must be 0 (joint) or 1 (per-level quota)")
+    for lo, hi, take in ranges:
+        f = np.arange(lo, hi, dtype=np.int64)
+        stream_f = np.concatenate([f, f])
+        stream_s = np.concatenate([qk[lo:hi], kq[lo:hi]]).astype(np.float64)
+        walk = stream_f[np.lexsort((stream_f, -stream_s))]
+        _, first = np.unique(walk, return_index=True)   # where each entry first shows up
+        flags[walk[np.sort(first)[:take]]] = True
     flags[C:] = True
     return flags
 
@@ -339,17 +354,17 @@ def pyramid_bwd(dxg: np.ndarray, slot_map: np.ndarray, N: int, L: int, p: int) -
 # --------------------------------------------------------------------------
 
 
-def forward_head(qh, kh, vh, L, p, k, scale=None, parity=True, flags=None):
+def forward_head(qh, kh, vh, L, p, k, scale=None, parity=True, flags=None, select_mode=0):
     """Forward of one (batch, head).  qh, kh, vh: [N, d] fp64.
 
     ``flags`` freezes the selection (used by gradient and causality checks).
     """
     N, d = qh.shape
-    check_config(N, L, p, k)
+    check_config(N, L, p, k, select_mode)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     qk, kq = scores(qh, kh, L, p)
     if flags is None:
-        flags = select(qk, kq, N, L, p, k)
+        flags = select(qk, kq, N, L, p, k, select_mode)
     sel_idx, slot_map = gather_order(flags, N, L, p)
     rnd = round_bf16 if parity else (lambda a: a)
     pyr = [pyramid(x, L, p) for x in (qh, kh, vh)]
@@ -381,7 +396,7 @@ def _head(x, b, h) -> np.ndarray:
     return np.ascontiguousarray(np.asarray(x[b, :, h, :], dtype=np.float64))
 
 
-def forward(q, k, v, L, p, kk, scale=None, parity=True):
+def forward(q, k, v, L, p, kk, scale=None, parity=True, select_mode=0):
     """Forward over every (b, h).  q, k, v: arrays [B, N, H, d] (any float
     dtype; converted exactly to fp64 per head).  Returns per-head states in a
     dict keyed by (b, h) and the output O [B, N, H, d]."""
@@ -391,7 +406,7 @@ def forward(q, k, v, L, p, kk, scale=None, parity=True):
     for b in range(B):
         for h in range(H):
             st = forward_head(_head(q, b, h), _head(k, b, h), _head(v, b, h),
-                              L, p, kk, scale, parity)
+                              L, p, kk, scale, parity, select_mode=select_mode)
             states[(b, h)] = st
             o[b, :, h, :] = st["o"]
     return o, states
@@ -412,11 +427,11 @@ def backward(states, do):
 # --------------------------------------------------------------------------
 
 
-def select_head(qh, kh, L, p, k):
+def select_head(qh, kh, L, p, k, select_mode=0):
     """Scores, flags, gather order and slot map of one head (no attention)."""
     N = qh.shape[0]
     qk, kq = scores(qh, kh, L, p)
-    flags = select(qk, kq, N, L, p, k)
+    flags = select(qk, kq, N, L, p, k, select_mode)
     sel_idx, slot_map = gather_order(flags, N, L, p)
     return dict(qk=qk, kq=kq, flags=flags, sel_idx=sel_idx, slot_map=slot_map)
 
