@@ -46,10 +46,15 @@ lh_status check(const lh_config* c) {
   if (c->k > (1LL << 31)) return LH_ERR_INVALID_ARGUMENT;
   const int64_t n_sel = (c->L - 1) * c->p * c->k;
   if (n_sel > cand) return LH_ERR_INVALID_ARGUMENT;
+  if (c->select_mode == 1 && c->L > 1) {   // p k must fit in the coarsest finer level
+    int64_t coarsest_finer = c->N;
+    for (int l = 0; l < c->L - 2; ++l) coarsest_finer /= c->p;
+    if ((int64_t)c->p * c->k > coarsest_finer) return LH_ERR_INVALID_ARGUMENT;
+  }
   if (P >= (1LL << 31)) return LH_ERR_UNSUPPORTED;
   if (c->d != 64 && c->d != 128) return LH_ERR_UNSUPPORTED;
   if (c->scatter_mode != 0 && c->scatter_mode != 1) return LH_ERR_INVALID_ARGUMENT;
-  if (c->select_mode != 0) return LH_ERR_UNSUPPORTED;
+  if (c->select_mode != 0 && c->select_mode != 1) return LH_ERR_UNSUPPORTED;
   if (!(c->scale == c->scale)) return LH_ERR_INVALID_ARGUMENT;
   const int64_t S = c->N / w + n_sel;
   if (S >= (1LL << 31) || (int64_t)c->B * c->H * ((S + 127) / 128) >= (1LL << 31))
@@ -77,6 +82,20 @@ LhDims dims(const lh_config* c) {
   D.n_cand = D.L > 1 ? D.lvl_off[D.L - 1] : 0;
   D.n_sel = (int64_t)(D.L - 1) * c->p * c->k;
   D.S = D.lvl_size[D.L - 1] + D.n_sel;
+  D.select_mode = c->select_mode;
+  if (c->select_mode == 1 && D.L > 1) {
+    D.nseg = D.L - 1;
+    for (int l = 0; l < D.L - 1; ++l) {
+      D.seg_lo[l] = D.lvl_off[l];
+      D.seg_len[l] = D.lvl_size[l];
+    }
+    D.seg_need = (int64_t)c->p * c->k;
+  } else {
+    D.nseg = 1;
+    D.seg_lo[0] = 0;
+    D.seg_len[0] = D.n_cand;
+    D.seg_need = D.n_sel;
+  }
   D.scale = c->scale > 0.f ? c->scale : (float)(1.0 / sqrt((double)c->d));
   D.status = nullptr;
   return D;

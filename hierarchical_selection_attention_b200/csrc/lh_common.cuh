@@ -23,6 +23,13 @@ struct LhDims {
   int64_t lvl_span[LH_MAX_LEVELS];   // p^l
   int64_t pool_row[LH_MAX_LEVELS];   // first pooled row of level l (l >= 1), per batch row
   int64_t pooled_rows;               // sum_{l>=1} N / p^l
+  // Selection segments: select_mode 0 has one (all finer entries, n_sel to
+  // take), select_mode 1 one per finer level (p k to take from each).
+  int select_mode;
+  int nseg;
+  int64_t seg_lo[LH_MAX_LEVELS];     // first flat index of segment s
+  int64_t seg_len[LH_MAX_LEVELS];    // its entries
+  int64_t seg_need;                  // entries to take from each segment
   float scale;
   int* status;                       // device status word [code, detail]
 };

@@ -16,6 +16,11 @@
 // selected(f) <=> key(f) >= threshold: integer work only, so the selected
 // set is bit-exact and the same on every run.
 //
+// Selection modes.  Mode 0 runs that selection once over all finer entries
+// (n_sel to take); mode 1, the per-level quota, runs it once per finer level
+// (p k to take from each, Eq. 8 read as an exact per-level count).  Each run
+// is a "segment" with its own histograms, state and threshold.
+//
 // Order.  Entries are sorted by the last base token they summarise,
 // e = (i+1) p^l - 1, and by level.  Walking the base tokens t in order and,
 // for each, the levels whose entries end at t ((t+1) mod p^l == 0) in
@@ -57,10 +62,12 @@ __global__ void __launch_bounds__(256) k_sel_hist(LhDims D, const float* __restr
                                                   const float* __restrict__ kq,
                                                   unsigned* __restrict__ hist,
                                                   const SelState* __restrict__ state, int pass) {
-  const int64_t bh = blockIdx.y;
+  const int64_t bs = blockIdx.y;                // (b, h) x segment
+  const int64_t bh = bs / D.nseg;
+  const int seg = (int)(bs - bh * D.nseg);
   unsigned long long prefix = 0;
   if (pass > 0) {
-    const SelState s = state[bh];
+    const SelState s = state[bs];
     if (s.done) return;
     prefix = s.prefix;
   }
@@ -72,9 +79,10 @@ __global__ void __launch_bounds__(256) k_sel_hist(LhDims D, const float* __restr
   const unsigned mask = (1u << c_width[pass]) - 1u;
   const float* q = qk + bh * D.P;
   const float* k = kq + bh * D.P;
-  const int64_t per_block = (D.n_cand + gridDim.x - 1) / gridDim.x;
-  const int64_t lo = (int64_t)blockIdx.x * per_block;
-  const int64_t end = min(lo + per_block, D.n_cand);
+  const int64_t seg_end = D.seg_lo[seg] + D.seg_len[seg];
+  const int64_t per_block = (D.seg_len[seg] + gridDim.x - 1) / gridDim.x;
+  const int64_t lo = D.seg_lo[seg] + (int64_t)blockIdx.x * per_block;
+  const int64_t end = min(lo + per_block, seg_end);
   const int64_t span = end > lo ? end - lo : 0;
   const int64_t rounds = (span + blockDim.x - 1) / blockDim.x;
   for (int64_t r = 0; r < rounds; ++r) {
@@ -94,20 +102,21 @@ __global__ void __launch_bounds__(256) k_sel_hist(LhDims D, const float* __restr
     }
   }
   __syncthreads();
-  unsigned* g = hist + (bh * kPasses + pass) * kBins;
+  unsigned* g = hist + (bs * kPasses + pass) * kBins;
   for (int i = threadIdx.x; i < kBins; i += blockDim.x)
     if (h[i]) atomicAdd(&g[i], h[i]);
 }
 
-// One block of 256 threads per (b, h); thread t owns digits 2047-8t .. 2040-8t.
+// One block of 256 threads per (b, h) and segment; thread t owns digits
+// 2047-8t .. 2040-8t.
 __global__ void __launch_bounds__(256) k_sel_find(LhDims D, const unsigned* __restrict__ hist,
                                                   SelState* __restrict__ state, int pass) {
-  const int64_t bh = blockIdx.x;
+  const int64_t bh = blockIdx.x;                 // (b, h) x segment
   SelState s;
   if (pass == 0) {
     s.prefix = 0;
-    s.need = D.n_sel;
-    s.done = D.n_sel == 0;
+    s.need = D.seg_need;
+    s.done = D.seg_need == 0;
     s.pad = 0;
     if (s.done) s.prefix = ~0ull;  // nothing is selected
   } else {
@@ -146,14 +155,16 @@ __global__ void __launch_bounds__(256) k_sel_find(LhDims D, const unsigned* __re
   }
 }
 
+// thr: the (b, h)'s segment states; an entry of level l < L-1 is compared with
+// the threshold of its segment (segment 0 in mode 0, segment l in mode 1).
 __device__ __forceinline__ bool selected_entry(const LhDims& D, const float* q, const float* k,
-                                               unsigned long long thr, int l, int64_t f) {
-  return (l == D.L - 1) || (entry_key(q, k, f) >= thr);
+                                               const SelState* thr, int l, int64_t f) {
+  return (l == D.L - 1) || (entry_key(q, k, f) >= thr[D.nseg > 1 ? l : 0].prefix);
 }
 
 // Number of selected entries that end on token t.
 __device__ __forceinline__ int count_at(const LhDims& D, const float* q, const float* k,
-                                        unsigned long long thr, int64_t t) {
+                                        const SelState* thr, int64_t t) {
   int n = 0;
   const uint32_t t1 = (uint32_t)(t + 1);  // N < 2^31
   for (int l = 0; l < D.L; ++l) {
@@ -169,7 +180,7 @@ __global__ void __launch_bounds__(kOrderThreads) k_order_count(LhDims D, const f
                                                               const SelState* __restrict__ state,
                                                               int* __restrict__ blk_cnt, int nblk) {
   const int64_t bh = blockIdx.y;
-  const unsigned long long thr = state[bh].prefix;
+  const SelState* thr = state + bh * D.nseg;
   const float* q = qk + bh * D.P;
   const float* k = kq + bh * D.P;
   const int64_t t0 = (int64_t)blockIdx.x * kOrderTile;
@@ -213,7 +224,7 @@ __global__ void __launch_bounds__(kOrderThreads) k_order_emit(LhDims D, const fl
                                                              int32_t* __restrict__ sel_idx,
                                                              int32_t* __restrict__ slot_map) {
   const int64_t bh = blockIdx.y;
-  const unsigned long long thr = state[bh].prefix;
+  const SelState* thr = state + bh * D.nseg;
   const float* q = qk + bh * D.P;
   const float* k = kq + bh * D.P;
   // each thread owns kOrderItems consecutive tokens so the scan order is t order
@@ -255,9 +266,10 @@ inline int64_t order_blocks(const LhDims& D) { return (D.N + kOrderTile - 1) / k
 
 size_t lh_select_ws_bytes(const LhDims& D) {
   const int64_t BH = (int64_t)D.B * D.H;
+  const int64_t BS = BH * D.nseg;
   size_t b = 0;
-  b += (size_t)BH * kPasses * kBins * sizeof(unsigned);
-  b += (size_t)BH * sizeof(SelState);
+  b += (size_t)BS * kPasses * kBins * sizeof(unsigned);
+  b += (size_t)BS * sizeof(SelState);
   b = (b + 255) & ~(size_t)255;
   b += (size_t)BH * order_blocks(D) * sizeof(int);
   return (b + 255) & ~(size_t)255;
@@ -267,27 +279,28 @@ cudaError_t lh_launch_select(const LhDims& D, const float* qk, const float* kq,
                              int32_t* sel_idx, int32_t* slot_map, void* ws, cudaStream_t st,
                              int* launches) {
   const int64_t BH = (int64_t)D.B * D.H;
+  const int64_t BS = BH * D.nseg;                 // (b, h) x selection segment
   unsigned* hist = reinterpret_cast<unsigned*>(ws);
-  SelState* state = reinterpret_cast<SelState*>(hist + BH * kPasses * kBins);
-  size_t off = (size_t)BH * kPasses * kBins * sizeof(unsigned) + (size_t)BH * sizeof(SelState);
+  SelState* state = reinterpret_cast<SelState*>(hist + BS * kPasses * kBins);
+  size_t off = (size_t)BS * kPasses * kBins * sizeof(unsigned) + (size_t)BS * sizeof(SelState);
   off = (off + 255) & ~(size_t)255;
   int* blk = reinterpret_cast<int*>(reinterpret_cast<char*>(ws) + off);
   const int nblk = (int)order_blocks(D);
   int n = 0;
-  cudaError_t e = cudaMemsetAsync(hist, 0, (size_t)BH * kPasses * kBins * sizeof(unsigned), st);
+  cudaError_t e = cudaMemsetAsync(hist, 0, (size_t)BS * kPasses * kBins * sizeof(unsigned), st);
   if (e != cudaSuccess) return e;
   if (D.n_cand > 0) {
     // ~8 candidates per thread per block keeps every SM busy on one head too
-    int64_t per = (D.n_cand + 148 * 4 - 1) / (148 * 4);
+    int64_t per = (D.seg_len[0] + 148 * 4 - 1) / (148 * 4);   // segment 0 is the largest
     per = per < 2048 ? 2048 : per;
-    const unsigned gx = (unsigned)((D.n_cand + per - 1) / per);
+    const unsigned gx = (unsigned)((D.seg_len[0] + per - 1) / per);
     for (int pass = 0; pass < kPasses; ++pass) {
-      k_sel_hist<<<dim3(gx, (unsigned)BH), 256, 0, st>>>(D, qk, kq, hist, state, pass);
-      k_sel_find<<<(unsigned)BH, 256, 0, st>>>(D, hist, state, pass);
+      k_sel_hist<<<dim3(gx, (unsigned)BS), 256, 0, st>>>(D, qk, kq, hist, state, pass);
+      k_sel_find<<<(unsigned)BS, 256, 0, st>>>(D, hist, state, pass);
       n += 2;
     }
   } else {
-    k_sel_find<<<(unsigned)BH, 256, 0, st>>>(D, hist, state, 0);
+    k_sel_find<<<(unsigned)BS, 256, 0, st>>>(D, hist, state, 0);
     n += 1;
   }
   k_order_count<<<dim3(nblk, (unsigned)BH), kOrderThreads, 0, st>>>(D, qk, kq, state, blk, nblk);

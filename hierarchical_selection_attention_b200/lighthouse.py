@@ -87,8 +87,9 @@ EXPORTED = ("lh_config_check", "lh_subseq_len", "lh_total_entries", "lh_pooled_r
             "lh_forward_launches", "lh_backward_launches")
 
 
-def make_config(B, N, H, d, L, p, k, scale: float = 0.0, scatter_mode: int = 0) -> lh_config:
-    return lh_config(B, N, H, d, L, p, k, scale, scatter_mode, 0)
+def make_config(B, N, H, d, L, p, k, scale: float = 0.0, scatter_mode: int = 0,
+                select_mode: int = 0) -> lh_config:
+    return lh_config(B, N, H, d, L, p, k, scale, scatter_mode, select_mode)
 
 
 def _ck(code: int, where: str):
@@ -287,8 +288,8 @@ class LighthouseLayer:
     """
 
     def __init__(self, B, N, H, d, L, p, k, scale: float = 0.0, scatter_mode: int = 0,
-                 device="cuda"):
-        self.cfg = make_config(B, N, H, d, L, p, k, scale, scatter_mode)
+                 device="cuda", select_mode: int = 0):
+        self.cfg = make_config(B, N, H, d, L, p, k, scale, scatter_mode, select_mode)
         _ck(lh_config_check(self.cfg), "lh_config_check")
         fwd, bwd, saved = lh_workspace_bytes(self.cfg)
         self.device = torch.device(device)

@@ -65,7 +65,11 @@ typedef enum {
  * not exceed the finer-level entry count.  scale <= 0 selects 1/sqrt(d).
  * scatter_mode: 0 = gather-side (pull) scatter; 1 = fixed-point integer
  * atomic scatter (same placement, order-independent sums).
- * select_mode: 0 = one joint top-k over all finer levels (the only mode). */
+ * select_mode: 0 = one joint top-k over all finer levels (Sec. 3.4);
+ *   1 = per-level quota: each of the L-1 finer levels contributes exactly
+ *   p k entries (the Eq. 8 accounting read literally), chosen within the
+ *   level by the same key order; needs p k <= N / p^(L-2).  S is the same in
+ *   both modes.  Other values: LH_ERR_UNSUPPORTED. */
 typedef struct {
   int64_t B, N, H, d, L, p, k;
   float scale;

@@ -77,3 +77,26 @@ def test_launch_counts(L):
     assert L.lh_forward_launches(cfg) > 5
     assert L.lh_backward_launches(cfg) >= 3
     assert L.lh_forward_launches(L.make_config(1, 100, 2, 64, 3, 4, 1)) == -1
+
+
+@pytest.mark.parametrize("mode,N,L_,p,k,code", [
+    (1, 4096, 3, 4, 64, 0),     # per-level quota: p k = 256 <= N / p = 1024
+    (1, 64, 3, 4, 4, 0),        # p k = 16 == the coarsest finer level
+    (1, 64, 3, 4, 5, 1),        # p k = 20 > 16 (the joint mode accepts it)
+    (0, 64, 3, 4, 5, 0),
+    (2, 4096, 3, 4, 64, 2),     # no stratified mode
+    (1, 640, 1, 4, 0, 0),       # one level: nothing to select in either mode
+])
+def test_select_mode_config(L, mode, N, L_, p, k, code):
+    cfg = L.make_config(1, N, 2, 64, L_, p, k, select_mode=mode)
+    assert L.lh_config_check(cfg) == code
+    if code == 0:
+        # S does not depend on the selection mode
+        assert L.lh_subseq_len(cfg) == lo.subseq_len(N, L_, p, k)
+
+
+def test_quota_mode_needs_a_larger_selection_workspace(L):
+    # one radix-selection state per finer level instead of one per head
+    f0, _, _ = L.lh_workspace_bytes(L.make_config(1, 4096, 2, 64, 3, 4, 64))
+    f1, _, _ = L.lh_workspace_bytes(L.make_config(1, 4096, 2, 64, 3, 4, 64, select_mode=1))
+    assert f1 > f0
