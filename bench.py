@@ -435,6 +435,71 @@ def run_reference(args, w):
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_sweep(args):
+    """Layer latency over sequence lengths (the paper's single-layer latency
+    figure): B=1, H=8, d=128, L=3, p=4, k = N/128 (1:64 sparsity), N from 8K
+    to 512K.  Forward and forward+backward through LighthouseLayer, CUDA
+    events on the launch stream, 3 warm-up and 10 timed runs each (median).
+    torch's causal scaled_dot_product_attention on the same Q, K, V is timed
+    beside it as context only (fewer runs at the longest lengths)."""
+    import torch.nn.functional as F
+    from hierarchical_selection_attention_b200 import lighthouse as L
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def med_ms(fn, reps, warm):
+        for _ in range(warm):
+            fn()
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    for N in [8192 << i for i in range(7)]:
+        B, H, d, Lv, p, k = 1, 8, 128, 3, 4, N // 128
+        q, kk, v = (t.to(dev) for t in make_qkv(B, N, H, d, seed=0))
+        dout = make_dout(B, N, H, d, seed=0).to(dev)
+        layer = L.LighthouseLayer(B, N, H, d, Lv, p, k, device=dev)
+        o = torch.empty_like(q)
+        grads = tuple(torch.empty_like(q) for _ in range(3))
+        fwd = med_ms(lambda: layer.forward(q, kk, v, out=o), 10, 3)
+        both = med_ms(lambda: (layer.forward(q, kk, v, out=o), layer.backward(dout, grads=grads)), 10, 3)
+        L.check_device_status()
+        line = {"N": N, "config": f"B=1 H=8 d=128 L=3 p=4 k={k} S={layer.S}",
+                "lighthouse_fwd_ms": round(fwd, 3), "lighthouse_fwd_bwd_ms": round(both, 3),
+                "lighthouse_fwd_tokens_per_s": B * N / (fwd / 1e3),
+                "lighthouse_fwd_bwd_tokens_per_s": B * N / (both / 1e3)}
+        if not args.no_sdpa:
+            # context only: dense causal attention over all N tokens, [B, H, N, d] views
+            try:
+                qt, kt, vt = (x.permute(0, 2, 1, 3).detach().requires_grad_() for x in (q, kk, v))
+                reps = 10 if N <= 65536 else 3
+                dense_fwd = med_ms(lambda: F.scaled_dot_product_attention(qt, kt, vt, is_causal=True),
+                                   reps, 2)
+
+                def dense_step():
+                    y = F.scaled_dot_product_attention(qt, kt, vt, is_causal=True)
+                    y.backward(dout.permute(0, 2, 1, 3))
+                dense_both = med_ms(dense_step, reps, 2)
+                line.update({"sdpa_causal_fwd_ms": round(dense_fwd, 3),
+                             "sdpa_causal_fwd_bwd_ms": round(dense_both, 3),
+                             "speedup_fwd": round(dense_fwd / fwd, 2),
+                             "speedup_fwd_bwd": round(dense_both / both, 2)})
+                del qt, kt, vt
+            except RuntimeError as e:   # no dense kernel for this shape on this build
+                line["sdpa_causal"] = f"unavailable: {str(e).splitlines()[0][:120]}"
+
+        print(json.dumps(line), flush=True)
+        del layer, q, kk, v, dout, o, grads
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -446,8 +511,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=32)
     ap.add_argument("--cpu-rows", type=int, default=96)
+    ap.add_argument("--sweep", action="store_true",
+                    help="latency over N = 8K..512K (one JSON line per N) instead of the bench line")
+    ap.add_argument("--no-sdpa", action="store_true", help="--sweep without the dense SDPA context")
     args = ap.parse_args()
     w = WORKLOADS[args.workload]
+    if args.sweep:
+        run_sweep(args)
+        return
 
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
