@@ -417,6 +417,36 @@ lh_status lh_backward(const lh_config* cfg, const void* saved, size_t saved_byte
   return cu(lh_launch_gather_bwd(D, dqg, dkg, dvg, slot_map, dq, dk, dv, st));
 }
 
+size_t lh_gemm_ws_bytes(int64_t M, int64_t N, int32_t splits) {
+  if (M < 1 || N < 1 || splits < 1) return 0;
+  return lh_gemm_partial_bytes(M, N, splits);
+}
+
+lh_status lh_gemm(int64_t M, int64_t N, int32_t npairs, const lh_gemm_operand* ops, int32_t a_mn,
+                  int32_t b_mn, lh_bf16* c, int64_t ldc, int32_t splits, void* ws,
+                  size_t ws_bytes, void* stream) {
+  if (!ops || !c || npairs < 1 || npairs > 3 || M < 1 || N < 1 || splits < 1) return LH_ERR_INVALID_ARGUMENT;
+  if (M >= (1LL << 31) || N >= (1LL << 31) || (N % 8) || ldc < N || (ldc % 8)) return LH_ERR_INVALID_ARGUMENT;
+  if ((a_mn != 0 && a_mn != 1) || (b_mn != 0 && b_mn != 1)) return LH_ERR_INVALID_ARGUMENT;
+  if (!all_aligned(c)) return LH_ERR_INVALID_ARGUMENT;
+  int64_t total = 0;
+  for (int i = 0; i < npairs; ++i) {
+    const lh_gemm_operand& o = ops[i];
+    if (!o.a || !o.b || o.k < 1 || (o.k % 8) || o.k >= (1LL << 31)) return LH_ERR_INVALID_ARGUMENT;
+    if (!all_aligned(o.a, o.b) || (o.lda % 8) || (o.ldb % 8)) return LH_ERR_INVALID_ARGUMENT;
+    if (o.lda < (a_mn ? M : o.k) || o.ldb < (b_mn ? N : o.k)) return LH_ERR_INVALID_ARGUMENT;
+    total += (o.k + 63) / 64;
+  }
+  if (splits > total) splits = (int32_t)total;
+  if (splits > 1 && (!ws || ws_bytes < lh_gemm_partial_bytes(M, N, splits) || !all_aligned(ws)))
+    return LH_ERR_WORKSPACE;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return cu(lh_launch_gemm(M, N, npairs, ops, a_mn, b_mn, c, ldc, splits, ws, status_ptr(), sms,
+                           (cudaStream_t)stream, nullptr));
+}
+
 lh_status lh_get_device_status(void* stream, int32_t* detail) {
   int* p = status_ptr();
   if (!p) return LH_ERR_CUDA;

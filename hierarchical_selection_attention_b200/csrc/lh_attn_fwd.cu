@@ -344,6 +344,9 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 
 }  // namespace
 
+// cuTensorMapEncodeTiled from the driver, looked up once.
+PFN_cuTensorMapEncodeTiled_v12000 lh_tensormap_encoder() { return get_encode(); }
+
 // Tensor map over a [BH, rows, d] bf16 tensor, box = 64 features x box_rows
 // rows of one (b, h), 128-byte swizzle; rows past `rows` read as zero.
 bool lh_make_tmap_3d(CUtensorMap* m, const void* base, int64_t BH, int64_t rows, int d,

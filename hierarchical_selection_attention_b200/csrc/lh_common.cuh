@@ -97,3 +97,10 @@ cudaError_t lh_launch_attn_bwd(int BH, int64_t S, int d, float scale, const lh_b
                                const float* lse, const float* delta, lh_bf16* dqg,
                                lh_bf16* dkg, lh_bf16* dvg, int* status, cudaStream_t st,
                                int which);
+
+// Plain GEMM (lh_gemm.cu).
+size_t lh_gemm_partial_bytes(int64_t M, int64_t N, int splits);
+cudaError_t lh_launch_gemm(int64_t M, int64_t N, int npairs, const lh_gemm_operand* ops, int a_mn,
+                           int b_mn, lh_bf16* c, int64_t ldc, int splits, void* ws, int* status,
+                           int num_sms, cudaStream_t st, int* launches);
+

@@ -18,6 +18,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liblighthouse.so")
 
 LH_OK = 0
+LH_ERR_INVALID_ARGUMENT = 1
 _STATUS = {0: "LH_OK", 1: "LH_ERR_INVALID_ARGUMENT", 2: "LH_ERR_UNSUPPORTED",
            3: "LH_ERR_WORKSPACE", 4: "LH_ERR_CUDA", 5: "LH_ERR_DEVICE_TIMEOUT",
            6: "LH_ERR_DEVICE_BOUNDS"}
@@ -37,6 +38,11 @@ class lh_config(ctypes.Structure):
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}
+
+
+class lh_gemm_operand(ctypes.Structure):
+    _fields_ = [("a", ctypes.c_void_p), ("b", ctypes.c_void_p), ("k", ctypes.c_int64),
+                ("lda", ctypes.c_int64), ("ldb", ctypes.c_int64)]
 
 
 def _load():
@@ -71,6 +77,9 @@ def _load():
         "lh_status_string": (ctypes.c_char_p, [I32]),
         "lh_forward_launches": (I32, [C]),
         "lh_backward_launches": (I32, [C]),
+        "lh_gemm_ws_bytes": (SZ, [I64, I64, I32]),
+        "lh_gemm": (I32, [I64, I64, I32, ctypes.POINTER(lh_gemm_operand), I32, I32, P, I64, I32, P,
+                          SZ, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -84,7 +93,7 @@ EXPORTED = ("lh_config_check", "lh_subseq_len", "lh_total_entries", "lh_pooled_r
             "lh_score_topk_noalloc", "lh_score_topk_noalloc_max_bytes", "lh_gather",
             "lh_attn_fwd", "lh_attn_bwd", "lh_attn_bwd_dkdv", "lh_attn_bwd_dq", "lh_scatter", "lh_scatter_bwd", "lh_gather_bwd",
             "lh_forward", "lh_backward", "lh_get_device_status", "lh_status_string",
-            "lh_forward_launches", "lh_backward_launches")
+            "lh_forward_launches", "lh_backward_launches", "lh_gemm_ws_bytes", "lh_gemm")
 
 
 def make_config(B, N, H, d, L, p, k, scale: float = 0.0, scatter_mode: int = 0,
@@ -278,6 +287,30 @@ def saved_views(cfg: lh_config, saved: torch.Tensor) -> dict:
                 qg=view(2, BF16, (B, H, S, d)), kg=view(3, BF16, (B, H, S, d)),
                 vg=view(4, BF16, (B, H, S, d)), og=view(5, BF16, (B, H, S, d)),
                 og_lo=view(6, BF16, (B, H, S, d)), lse=view(7, F32, (B, H, S)))
+
+
+def lh_gemm_ws_bytes(M, N, splits=1):
+    return int(_lib.lh_gemm_ws_bytes(M, N, splits))
+
+
+def lh_gemm(c, pairs, a_mn=0, b_mn=0, splits=1, ws=None, stream=None):
+    """C[M, N] = sum_i A_i B_i^T into the bf16 matrix c (row-major, may be a
+    row-slice view with its own stride).  pairs: list of (a, b, k) with a, b
+    bf16 2-D tensors; a is [M, k] (a_mn=0) or [k, M] (a_mn=1), b is [N, k]
+    (b_mn=0) or [k, N] (b_mn=1), each with unit inner stride."""
+    M, N = c.shape
+    ops = (lh_gemm_operand * len(pairs))()
+    for i, (a, b, k) in enumerate(pairs):
+        for t in (a, b):
+            if t.dtype != BF16 or t.dim() != 2 or t.stride(1) != 1 or not t.is_cuda:
+                raise LighthouseError(LH_ERR_INVALID_ARGUMENT, "lh_gemm operand")
+        ops[i] = lh_gemm_operand(a.data_ptr(), b.data_ptr(), k, a.stride(0), b.stride(0))
+    if c.dtype != BF16 or c.stride(1) != 1:
+        raise LighthouseError(LH_ERR_INVALID_ARGUMENT, "lh_gemm output")
+    nb = 0 if ws is None else ws.numel() * ws.element_size()
+    _ck(_lib.lh_gemm(M, N, len(pairs), ops, a_mn, b_mn, c.data_ptr(), c.stride(0), splits,
+                     _p(ws), nb, _stream(stream)), "lh_gemm")
+    return c
 
 
 class LighthouseLayer:

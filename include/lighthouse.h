@@ -240,6 +240,34 @@ lh_status lh_backward(const lh_config* cfg, const void* saved, size_t saved_byte
                       const lh_bf16* dout, lh_bf16* dq, lh_bf16* dk, lh_bf16* dv,
                       void* ws, size_t ws_bytes, void* stream);
 
+/* ---- plain GEMMs for the projections around the layer (Sec. 3.1: per-head
+ * Q, K, V come from the layer's own W_Q, W_K, W_V; an output projection
+ * follows).  Not part of the pages' custom kernels: the pages leave these to
+ * the training framework; they are here so a whole layer can be timed.
+ *
+ *   C[M, N] = sum_{i < npairs} A_i[M, K_i] B_i[N, K_i]^T
+ *
+ * bf16 in, fp32 accumulate, bf16 out (C row-major, leading dimension ldc).
+ * a_mn = 0: A_i[m, k] at a + m * lda + k (K contiguous); a_mn = 1: at
+ * a + k * lda + m (M contiguous).  Likewise b_mn for B_i with n.  npairs in
+ * 1..3; M, N, K_i >= 1; N, K_i, lda, ldb, ldc multiples of 8; pointers
+ * 16-byte aligned; lda >= K_i (a_mn = 0) or M (a_mn = 1), ldb likewise.
+ * splits > 1 divides the summed K range over CTAs (for long K and few
+ * output tiles) and needs `ws` of lh_gemm_ws_bytes bytes for fp32 partials,
+ * summed afterwards in split order, so the result is deterministic.
+ * Invalid arguments return LH_ERR_INVALID_ARGUMENT before any launch. */
+typedef struct {
+  const lh_bf16* a;
+  const lh_bf16* b;
+  int64_t k, lda, ldb;
+} lh_gemm_operand;
+
+size_t lh_gemm_ws_bytes(int64_t M, int64_t N, int32_t splits);
+
+lh_status lh_gemm(int64_t M, int64_t N, int32_t npairs, const lh_gemm_operand* ops, int32_t a_mn,
+                  int32_t b_mn, lh_bf16* c, int64_t ldc, int32_t splits, void* ws,
+                  size_t ws_bytes, void* stream);
+
 /* Synchronises `stream`, returns the first device-side error recorded since
  * the last call (LH_OK if none) and clears it.  *detail (may be NULL)
  * receives a kernel-specific code locating the failure. */
