@@ -466,3 +466,51 @@ def outputs_at(qh, kh, vh, L, p, k, t_list, scale=None, parity=True, sel=None):
         for s in need.get(int(t), []):          # ascending level order
             out[n] += og_rows[pos[s]]
     return out, dict(sel=sel, rows=rows, og=og_rows, lse=lse_rows, qg=qg, kg=kg, vg=vg)
+
+
+# --------------------------------------------------------------------------
+# The projections on either side of the layer (Sec. 3.1): per-head Q, K, V
+# come from the layer's own W_Q, W_K, W_V, and the output projection W_O
+# follows.  Plain products; the library computes them with its own GEMM.
+# --------------------------------------------------------------------------
+
+
+def projected_forward(x, wq, wk, wv, wo, H, L, p, k, scale=None, parity=True, select_mode=0,
+                      flags=None):
+    """x [B, N, Dm]; wq, wk, wv [H d, Dm]; wo [Dm, H d].
+
+    Q = x wq^T, K = x wk^T, V = x wv^T (split into H heads of d), the
+    Lighthouse layer per head, y = O wo^T.  Parity mode rounds to bf16 where
+    the library stores bf16 (Q, K, V, O, y).  ``flags`` ({(b, h): flags})
+    freezes the selection."""
+    B, N, Dm = x.shape
+    rnd = round_bf16 if parity else (lambda a: a)
+    q, kk, v = (rnd(x @ w.T).reshape(B, N, H, -1) for w in (wq, wk, wv))
+    o = np.zeros_like(q)
+    states = {}
+    for b in range(B):
+        for h in range(H):
+            st = forward_head(_head(q, b, h), _head(kk, b, h), _head(v, b, h), L, p, k, scale,
+                              parity, flags=None if flags is None else flags[(b, h)],
+                              select_mode=select_mode)
+            states[(b, h)] = st
+            o[b, :, h, :] = st["o"]
+    o = rnd(o)
+    y = rnd(o.reshape(B, N, -1) @ wo.T)
+    return y, dict(x=x, wq=wq, wk=wk, wv=wv, wo=wo, q=q, k=kk, v=v, o=o, states=states,
+                   parity=parity)
+
+
+def projected_backward(st, dy):
+    """Gradients (dx, dwq, dwk, dwv, dwo) of <y, dy>, the selection frozen."""
+    rnd = round_bf16 if st["parity"] else (lambda a: a)
+    x, o = st["x"], st["o"]
+    B, N, Dm = x.shape
+    do = rnd(dy @ st["wo"]).reshape(o.shape)
+    grads = backward(st["states"], do)
+    dq, dk, dv = (rnd(g).reshape(B * N, -1) for g in grads)
+    xf, of, dyf = x.reshape(B * N, Dm), o.reshape(B * N, -1), dy.reshape(B * N, -1)
+    dx = rnd(dq @ st["wq"] + dk @ st["wk"] + dv @ st["wv"]).reshape(B, N, Dm)
+    dwq, dwk, dwv = (rnd(g.T @ xf) for g in (dq, dk, dv))
+    dwo = rnd(dyf.T @ of)
+    return dx, dwq, dwk, dwv, dwo
