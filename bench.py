@@ -500,6 +500,59 @@ def run_sweep(args):
         torch.cuda.empty_cache()
 
 
+def run_full_layer(args, w):
+    """The layer with its projections (LighthouseProjectedLayer) on the bench
+    workload, d_model = H d: forward + backward tokens/s, and the share of
+    the step the Lighthouse layer itself takes.  Synthetic x, dy and weights
+    (N(0,1) x 1/sqrt(d_model), bf16)."""
+    from hierarchical_selection_attention_b200 import lighthouse as L
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    B, N, H, d, Lv, p, k = (w[x] for x in ("B", "N", "H", "d", "L", "p", "k"))
+    Dm = H * d
+    g = torch.Generator(device=dev).manual_seed(args.workload)
+    x = torch.randn(B, N, Dm, generator=g, device=dev).to(torch.bfloat16)
+    dy = torch.randn(B, N, Dm, generator=g, device=dev).to(torch.bfloat16)
+    ws_ = [(torch.randn(*s_, generator=g, device=dev) / math.sqrt(Dm)).to(torch.bfloat16)
+           for s_ in ((H * d, Dm),) * 3 + ((Dm, H * d),)]
+    layer = L.LighthouseProjectedLayer(B, N, H, d, Dm, Lv, p, k, device=dev)
+    y = torch.empty_like(x)
+    grads = (torch.empty_like(x), *(torch.empty_like(ws_[0]) for _ in range(3)), torch.empty_like(ws_[3]))
+
+    def step():
+        layer.forward(x, *ws_, y=y)
+        layer.backward(dy, grads=grads)
+
+    def core_step():
+        layer.core.forward(layer.q, layer.k, layer.v, out=layer.o)
+        layer.core.backward(layer.do, grads=(layer.dq, layer.dk, layer.dv))
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / args.steps
+
+    ms = timed(step)
+    core_ms = timed(core_step)
+    L.check_device_status()
+    gemm_flop = 2 * B * N * Dm * H * d * (4 + 7)   # fwd: Q, K, V, y; bwd: dO, dW_o, dx (3), dW (3)
+    gemm_ms = ms - core_ms
+    return {"metric": "Lighthouse layer with projections, fwd+bwd tokens/s (1 B200)",
+            "value": B * N / (ms / 1e3), "unit": UNIT, "ms_per_step": ms,
+            "lighthouse_core_ms": core_ms, "projections_ms": gemm_ms,
+            "projections_TFLOP/s": gemm_flop / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None,
+            "steps": args.steps, "warmup": args.warmup, "dtype": "bf16",
+            "config": {"workload": w["name"], "d_model": Dm}}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -514,10 +567,15 @@ def main():
     ap.add_argument("--sweep", action="store_true",
                     help="latency over N = 8K..512K (one JSON line per N) instead of the bench line")
     ap.add_argument("--no-sdpa", action="store_true", help="--sweep without the dense SDPA context")
+    ap.add_argument("--full-layer", action="store_true",
+                    help="time the layer with its Q/K/V/output projections (one JSON line)")
     args = ap.parse_args()
     w = WORKLOADS[args.workload]
     if args.sweep:
         run_sweep(args)
+        return
+    if args.full_layer:
+        print(json.dumps(run_full_layer(args, w)), flush=True)
         return
 
     if args.impl == "reference":

@@ -346,6 +346,68 @@ class LighthouseLayer:
         return saved_views(self.cfg, self.saved)
 
 
+class LighthouseProjectedLayer:
+    """The layer with its projections (Sec. 3.1): per-head Q, K, V from the
+    layer's own W_Q, W_K, W_V, the Lighthouse layer, the output projection:
+
+        y = Lighthouse(x W_q^T, x W_k^T, x W_v^T) W_o^T
+
+    x, y [B, N, Dm]; wq, wk, wv [H d, Dm]; wo [Dm, H d]; all bf16 and owned
+    by the caller.  forward(x, wq, wk, wv, wo) -> y and backward(dy) ->
+    (dx, dwq, dwk, dwv, dwo) run every product in lh_gemm and the layer in
+    lh_forward / lh_backward, on torch's current stream.
+    """
+
+    def __init__(self, B, N, H, d, Dm, L, p, k, scale: float = 0.0, device="cuda",
+                 select_mode: int = 0):
+        self.core = LighthouseLayer(B, N, H, d, L, p, k, scale, device=device,
+                                    select_mode=select_mode)
+        self.shape = (B, N, H, d, Dm)
+        dev = self.core.device
+        e = lambda *s: torch.empty(*s, dtype=BF16, device=dev)
+        self.q, self.k, self.v, self.o = (e(B, N, H, d) for _ in range(4))
+        self.do, self.dq, self.dk, self.dv = (e(B, N, H, d) for _ in range(4))
+        # weight gradients: K = B N is long and there are few output tiles,
+        # so the K range is split over enough CTAs to fill the GPU
+        tiles = -(-(H * d) // 128) * -(-Dm // 256)
+        self.wsplits = max(1, min(16, 2 * 148 // max(1, tiles)))
+        nbytes = max(lh_gemm_ws_bytes(H * d, Dm, self.wsplits), lh_gemm_ws_bytes(Dm, H * d, self.wsplits))
+        self.gemm_ws = torch.empty(max(1, nbytes), dtype=torch.uint8, device=dev)
+
+    def forward(self, x, wq, wk, wv, wo, y=None):
+        B, N, H, d, Dm = self.shape
+        T, HD = B * N, H * d
+        x2 = x.view(T, Dm)
+        for dst, w in ((self.q, wq), (self.k, wk), (self.v, wv)):
+            lh_gemm(dst.view(T, HD), [(x2, w, Dm)])
+        self.core.forward(self.q, self.k, self.v, out=self.o)
+        y = torch.empty(B, N, Dm, dtype=BF16, device=x.device) if y is None else y
+        lh_gemm(y.view(T, Dm), [(self.o.view(T, HD), wo, HD)])
+        self._saved = (x, wq, wk, wv, wo)
+        return y
+
+    def backward(self, dy, grads=None):
+        B, N, H, d, Dm = self.shape
+        T, HD = B * N, H * d
+        x, wq, wk, wv, wo = self._saved
+        dev = dy.device
+        if grads is None:
+            grads = (torch.empty(B, N, Dm, dtype=BF16, device=dev),
+                     *(torch.empty(HD, Dm, dtype=BF16, device=dev) for _ in range(3)),
+                     torch.empty(Dm, HD, dtype=BF16, device=dev))
+        dx, dwq, dwk, dwv, dwo = grads
+        dy2 = dy.view(T, Dm)
+        lh_gemm(self.do.view(T, HD), [(dy2, wo, Dm)], b_mn=1)                  # dO = dy W_o
+        lh_gemm(dwo, [(dy2, self.o.view(T, HD), T)], a_mn=1, b_mn=1,           # dW_o = dy^T O
+                splits=self.wsplits, ws=self.gemm_ws)
+        self.core.backward(self.do, grads=(self.dq, self.dk, self.dv))
+        g = [t.view(T, HD) for t in (self.dq, self.dk, self.dv)]
+        lh_gemm(dx.view(T, Dm), [(g[0], wq, HD), (g[1], wk, HD), (g[2], wv, HD)], b_mn=1)
+        for dw, gi in zip((dwq, dwk, dwv), g):                                 # dW_i = dQ_i^T x
+            lh_gemm(dw, [(gi, x.view(T, Dm), T)], a_mn=1, b_mn=1, splits=self.wsplits, ws=self.gemm_ws)
+        return grads
+
+
 class LighthouseAttention(torch.autograd.Function):
     """Autograd wrapper: y = Lighthouse(q, k, v); the selection is not differentiated."""
 
