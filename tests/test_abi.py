@@ -100,3 +100,30 @@ def test_quota_mode_needs_a_larger_selection_workspace(L):
     f0, _, _ = L.lh_workspace_bytes(L.make_config(1, 4096, 2, 64, 3, 4, 64))
     f1, _, _ = L.lh_workspace_bytes(L.make_config(1, 4096, 2, 64, 3, 4, 64, select_mode=1))
     assert f1 > f0
+
+
+def test_gemm_argument_checks(L):
+    """lh_gemm rejects bad shapes and layouts before any launch (no GPU needed)."""
+    import ctypes
+    op = L.lh_gemm_operand
+    P = ctypes.c_void_p
+
+    def call(M, N, ops, c=0x1000, ldc=None, a_mn=0, b_mn=0, splits=1, ws=None, nb=0):
+        arr = (op * max(1, len(ops)))(*ops)
+        return L._lib.lh_gemm(M, N, len(ops), arr, a_mn, b_mn, P(c), N if ldc is None else ldc,
+                              splits, P(ws), nb, P(0))
+
+    ok_op = op(0x2000, 0x3000, 64, 64, 64)
+    assert call(128, 256, []) == 1                                   # no pairs
+    assert call(128, 250, [ok_op]) == 1                              # N not a multiple of 8
+    assert call(128, 256, [op(0x2000, 0x3000, 60, 64, 64)]) == 1     # K not a multiple of 8
+    assert call(128, 256, [op(0x2008, 0x3000, 64, 64, 64)]) == 1     # misaligned A
+    assert call(128, 256, [op(0x2000, 0x3000, 64, 32, 64)]) == 1     # lda < K (K-major A)
+    assert call(128, 256, [op(0x2000, 0x3000, 64, 64, 64)], a_mn=1) == 1   # lda < M (MN-major A)
+    assert call(128, 256, [ok_op], ldc=200) == 1                     # ldc < N
+    assert call(128, 256, [ok_op] * 4) == 1                          # more than three pairs
+    assert call(128, 256, [ok_op], a_mn=2) == 1                      # unknown layout
+    big = op(0x2000, 0x3000, 8192, 8192, 8192)
+    assert call(128, 256, [big], splits=4) == 3                      # split K without a workspace
+    assert L.lh_gemm_ws_bytes(128, 256, 4) == 4 * 128 * 256 * 4
+    assert L.lh_gemm_ws_bytes(128, 256, 1) == 0
