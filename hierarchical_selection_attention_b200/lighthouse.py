@@ -304,6 +304,9 @@ def lh_gemm(c, pairs, a_mn=0, b_mn=0, splits=1, ws=None, stream=None):
         for t in (a, b):
             if t.dtype != BF16 or t.dim() != 2 or t.stride(1) != 1 or not t.is_cuda:
                 raise LighthouseError(LH_ERR_INVALID_ARGUMENT, "lh_gemm operand")
+        # the kernel reads exactly these extents (the C ABI cannot see allocations)
+        if tuple(a.shape) != ((k, M) if a_mn else (M, k)) or tuple(b.shape) != ((k, N) if b_mn else (N, k)):
+            raise LighthouseError(LH_ERR_INVALID_ARGUMENT, "lh_gemm operand shape")
         ops[i] = lh_gemm_operand(a.data_ptr(), b.data_ptr(), k, a.stride(0), b.stride(0))
     if c.dtype != BF16 or c.stride(1) != 1:
         raise LighthouseError(LH_ERR_INVALID_ARGUMENT, "lh_gemm output")

@@ -255,7 +255,9 @@ lh_status lh_backward(const lh_config* cfg, const void* saved, size_t saved_byte
  * splits > 1 divides the summed K range over CTAs (for long K and few
  * output tiles) and needs `ws` of lh_gemm_ws_bytes bytes for fp32 partials,
  * summed afterwards in split order, so the result is deterministic.
- * Invalid arguments return LH_ERR_INVALID_ARGUMENT before any launch. */
+ * Invalid arguments return LH_ERR_INVALID_ARGUMENT before any launch.  The
+ * caller guarantees that every operand holds its full extent (M or N rows
+ * by K_i, at its leading dimension): the library cannot see allocations. */
 typedef struct {
   const lh_bf16* a;
   const lh_bf16* b;

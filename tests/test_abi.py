@@ -127,3 +127,15 @@ def test_gemm_argument_checks(L):
     assert call(128, 256, [big], splits=4) == 3                      # split K without a workspace
     assert L.lh_gemm_ws_bytes(128, 256, 4) == 4 * 128 * 256 * 4
     assert L.lh_gemm_ws_bytes(128, 256, 1) == 0
+
+
+def test_gemm_binding_checks_operand_shapes(L):
+    """The binding refuses operands whose extents differ from (M or N) x k, so
+    the kernel never reads past an allocation (CPU tensors fail the device
+    check first, the shape rule is the same)."""
+    import torch
+    c = torch.empty(128, 256, dtype=torch.bfloat16)
+    a = torch.empty(128, 64, dtype=torch.bfloat16)
+    b = torch.empty(256, 64, dtype=torch.bfloat16)
+    with pytest.raises(L.LighthouseError):
+        L.lh_gemm(c, [(a, b, 64)])      # host tensors are refused before any call
