@@ -76,43 +76,66 @@ __global__ void __launch_bounds__(kThreads) k_gather(LhDims D, const uint4* __re
   vg[o] = __ldg(level_row(D, v, v_lv, l, b, i, h, V) + cv);
 }
 
-// (iv) scatter-back, gather side: thread = (b, t, h, vector cv); the entry of
-// level l that reaches t is i = floor((t+1)/p^l) - 1.  All slot lookups are
-// issued before any row load, and all row loads before the sum, so a thread
-// waits for two memory round trips rather than two per level.
+// Tokens a thread of k_scatter / k_gather_bwd takes: G divides p (and N), so
+// the G tokens of an aligned group share their entry at every level l >= 1,
+// and each thread turns two memory round trips (slot lookups, then rows) into
+// G output rows instead of one.
+constexpr int kMaxG = 4;
+
+// (iv) scatter-back, gather side: thread = (b, group g, h, vector cv), where
+// group g holds the tokens t with t + 1 in [gG, gG + G).  The entry of level l
+// that reaches t is i = floor((t+1)/p^l) - 1, the same for the whole group at
+// every l >= 1; level 0 contributes entry t itself.  All slot lookups are
+// issued before any row load, and all row loads before the sums; each row is
+// summed in ascending level order.
 template <int L, typename I>
-__global__ void __launch_bounds__(kThreads) k_scatter(LhDims D, const uint4* __restrict__ og,
+__global__ void __launch_bounds__(kThreads) k_scatter(LhDims D, int G, I NG,
+                                                      const uint4* __restrict__ og,
                                                       const int32_t* __restrict__ slot_map,
                                                       uint4* __restrict__ o) {
+  constexpr int LC = L > 1 ? L - 1 : 1;
   const int V = D.d >> 3;
   const I item = (I)blockIdx.x * blockDim.x + threadIdx.x;
-  const I total = (I)D.B * D.N * D.H * V;
+  const I total = (I)D.B * NG * D.H * V;
   if (item >= total) return;
   const int cv = (int)(item & (V - 1));
-  const I r = item / V;  // (b, t, h)
+  const I r = item / V;  // (b, g, h)
   const int h = (int)(r % (I)D.H);
-  const I bt = r / (I)D.H;
-  const int64_t t = (int64_t)(bt % (I)D.N);
-  const int b = (int)(bt / (I)D.N);
+  const I bg = r / (I)D.H;
+  const int64_t j0 = (int64_t)(bg % NG) * G;  // t + 1 of the group's first token
+  const int b = (int)(bg / NG);
   const int64_t bh = (int64_t)b * D.H + h;
   const int32_t* sm = slot_map + bh * D.P;
   const uint4* src = og + bh * D.S * V + cv;
-  const uint32_t t1 = (uint32_t)(t + 1);
-  int slot[L];
+  int cslot[LC], fslot[kMaxG];
 #pragma unroll
-  for (int l = 0; l < L; ++l) {
-    const uint32_t j = t1 / (uint32_t)D.lvl_span[l];
-    slot[l] = j ? __ldg(sm + D.lvl_off[l] + j - 1) : -1;
+  for (int l = 1; l < L; ++l) {
+    const int64_t j = j0 / D.lvl_span[l];
+    cslot[l - 1] = j ? __ldg(sm + D.lvl_off[l] + j - 1) : -1;
   }
-  uint4 row[L];
 #pragma unroll
-  for (int l = 0; l < L; ++l)
-    if (slot[l] >= 0) row[l] = __ldg(src + (int64_t)slot[l] * V);
-  float a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (int u = 0; u < kMaxG; ++u) {
+    const int64_t t = j0 - 1 + u;
+    fslot[u] = (u < G && t >= 0 && t < D.N) ? __ldg(sm + D.lvl_off[0] + t) : -1;
+  }
+  uint4 crow[LC], frow[kMaxG];
 #pragma unroll
-  for (int l = 0; l < L; ++l)
-    if (slot[l] >= 0) acc8(a, row[l]);
-  o[item] = pack8(a);
+  for (int l = 1; l < L; ++l)
+    if (cslot[l - 1] >= 0) crow[l - 1] = __ldg(src + (int64_t)cslot[l - 1] * V);
+#pragma unroll
+  for (int u = 0; u < kMaxG; ++u)
+    if (fslot[u] >= 0) frow[u] = __ldg(src + (int64_t)fslot[u] * V);
+#pragma unroll
+  for (int u = 0; u < kMaxG; ++u) {
+    const int64_t t = j0 - 1 + u;
+    if (u >= G || t < 0 || t >= D.N) continue;
+    float a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (fslot[u] >= 0) acc8(a, frow[u]);
+#pragma unroll
+    for (int l = 1; l < L; ++l)
+      if (cslot[l - 1] >= 0) acc8(a, crow[l - 1]);
+    o[(((int64_t)b * D.N + t) * D.H + h) * V + cv] = pack8(a);
+  }
 }
 
 // (iv) in fixed-point integer atomics: every selected entry adds its output,
@@ -229,55 +252,78 @@ __global__ void __launch_bounds__(kThreads) k_attn_delta(int64_t rows, int V,
   if (item % V == 0) delta[item / V] = s;
 }
 
-// Adjoint of gather + mean pooling: thread = (b, t, h, vector cv); the level-l
-// entry whose (unshifted) window holds t is i = floor(t / p^l).  Slot lookups
-// first, then every row load, then the sums (two memory round trips).
+// Adjoint of gather + mean pooling: thread = (b, group g, h, vector cv),
+// group g holding the tokens t in [gG, gG + G).  The level-l entry whose
+// (unshifted) window holds t is i = floor(t / p^l), the same for the whole
+// group at every l >= 1.  Slot lookups first, then every row load, then the
+// sums, each in ascending level order (two memory round trips per G rows).
 template <int L, typename I>
-__global__ void __launch_bounds__(kThreads) k_gather_bwd(LhDims D, const uint4* __restrict__ dqg,
-                                                         const uint4* __restrict__ dkg,
-                                                         const uint4* __restrict__ dvg,
-                                                         const int32_t* __restrict__ slot_map,
-                                                         uint4* __restrict__ dq, uint4* __restrict__ dk,
-                                                         uint4* __restrict__ dv) {
+__global__ void __launch_bounds__(kThreads, L <= 4 ? 2 : 1)
+    k_gather_bwd(LhDims D, int G, I NG, const uint4* __restrict__ dqg,
+                 const uint4* __restrict__ dkg, const uint4* __restrict__ dvg,
+                 const int32_t* __restrict__ slot_map, uint4* __restrict__ dq,
+                 uint4* __restrict__ dk, uint4* __restrict__ dv) {
+  constexpr int LC = L > 1 ? L - 1 : 1;
   const int V = D.d >> 3;
   const I item = (I)blockIdx.x * blockDim.x + threadIdx.x;
-  const I total = (I)D.B * D.N * D.H * V;
+  const I total = (I)D.B * NG * D.H * V;
   if (item >= total) return;
   const int cv = (int)(item & (V - 1));
   const I r = item / V;
   const int h = (int)(r % (I)D.H);
-  const I bt = r / (I)D.H;
-  const int64_t t = (int64_t)(bt % (I)D.N);
-  const int b = (int)(bt / (I)D.N);
+  const I bg = r / (I)D.H;
+  const int64_t t0 = (int64_t)(bg % NG) * G;
+  const int b = (int)(bg / NG);
   const int64_t bh = (int64_t)b * D.H + h;
   const int32_t* sm = slot_map + bh * D.P;
-  int slot[L];
+  const int64_t base = bh * D.S * V + cv;
+  int cslot[LC], fslot[kMaxG];
 #pragma unroll
-  for (int l = 0; l < L; ++l)
-    slot[l] = __ldg(sm + D.lvl_off[l] + (uint32_t)t / (uint32_t)D.lvl_span[l]);
-  uint4 rq[L], rk[L], rv[L];
+  for (int l = 1; l < L; ++l) cslot[l - 1] = __ldg(sm + D.lvl_off[l] + t0 / D.lvl_span[l]);
 #pragma unroll
-  for (int l = 0; l < L; ++l) {
-    if (slot[l] >= 0) {
-      const int64_t s = (bh * D.S + slot[l]) * V + cv;
-      rq[l] = __ldg(dqg + s);
-      rk[l] = __ldg(dkg + s);
-      rv[l] = __ldg(dvg + s);
+  for (int u = 0; u < kMaxG; ++u) fslot[u] = u < G ? __ldg(sm + D.lvl_off[0] + t0 + u) : -1;
+  uint4 cq[LC], ck[LC], cvv[LC], fq[kMaxG], fk[kMaxG], fv[kMaxG];
+#pragma unroll
+  for (int l = 1; l < L; ++l) {
+    if (cslot[l - 1] >= 0) {
+      const int64_t s = base + (int64_t)cslot[l - 1] * V;
+      cq[l - 1] = __ldg(dqg + s);
+      ck[l - 1] = __ldg(dkg + s);
+      cvv[l - 1] = __ldg(dvg + s);
     }
   }
-  float aq[8] = {0, 0, 0, 0, 0, 0, 0, 0}, ak[8] = {0, 0, 0, 0, 0, 0, 0, 0},
-        av[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
-  for (int l = 0; l < L; ++l) {
-    if (slot[l] < 0) continue;
-    const float w = 1.f / (float)D.lvl_span[l];
-    acc8(aq, rq[l], w);
-    acc8(ak, rk[l], w);
-    acc8(av, rv[l], w);
+  for (int u = 0; u < kMaxG; ++u) {
+    if (fslot[u] >= 0) {
+      const int64_t s = base + (int64_t)fslot[u] * V;
+      fq[u] = __ldg(dqg + s);
+      fk[u] = __ldg(dkg + s);
+      fv[u] = __ldg(dvg + s);
+    }
   }
-  dq[item] = pack8(aq);
-  dk[item] = pack8(ak);
-  dv[item] = pack8(av);
+#pragma unroll
+  for (int u = 0; u < kMaxG; ++u) {
+    if (u >= G) continue;
+    float aq[8] = {0, 0, 0, 0, 0, 0, 0, 0}, ak[8] = {0, 0, 0, 0, 0, 0, 0, 0},
+          av[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (fslot[u] >= 0) {
+      acc8(aq, fq[u]);
+      acc8(ak, fk[u]);
+      acc8(av, fv[u]);
+    }
+#pragma unroll
+    for (int l = 1; l < L; ++l) {
+      if (cslot[l - 1] < 0) continue;
+      const float w = 1.f / (float)D.lvl_span[l];
+      acc8(aq, cq[l - 1], w);
+      acc8(ak, ck[l - 1], w);
+      acc8(av, cvv[l - 1], w);
+    }
+    const int64_t o = (((int64_t)b * D.N + t0 + u) * D.H + h) * V + cv;
+    dq[o] = pack8(aq);
+    dk[o] = pack8(ak);
+    dv[o] = pack8(av);
+  }
 }
 
 inline unsigned nblocks(int64_t n) { return (unsigned)((n + kThreads - 1) / kThreads); }
@@ -285,34 +331,41 @@ inline unsigned nblocks(int64_t n) { return (unsigned)((n + kThreads - 1) / kThr
 constexpr int64_t kIdx32 = (int64_t)1 << 31;  // item counts below this use 32-bit indices
 
 template <typename I>
-cudaError_t scatter_L(const LhDims& D, unsigned g, const uint4* x, const int32_t* sm, uint4* o,
-                      cudaStream_t st) {
+cudaError_t scatter_L(const LhDims& D, unsigned g, int G, I NG, const uint4* x, const int32_t* sm,
+                      uint4* o, cudaStream_t st) {
   switch (D.L) {
-    case 1: k_scatter<1, I><<<g, kThreads, 0, st>>>(D, x, sm, o); break;
-    case 2: k_scatter<2, I><<<g, kThreads, 0, st>>>(D, x, sm, o); break;
-    case 3: k_scatter<3, I><<<g, kThreads, 0, st>>>(D, x, sm, o); break;
-    case 4: k_scatter<4, I><<<g, kThreads, 0, st>>>(D, x, sm, o); break;
-    case 5: k_scatter<5, I><<<g, kThreads, 0, st>>>(D, x, sm, o); break;
-    case 6: k_scatter<6, I><<<g, kThreads, 0, st>>>(D, x, sm, o); break;
+    case 1: k_scatter<1, I><<<g, kThreads, 0, st>>>(D, G, NG, x, sm, o); break;
+    case 2: k_scatter<2, I><<<g, kThreads, 0, st>>>(D, G, NG, x, sm, o); break;
+    case 3: k_scatter<3, I><<<g, kThreads, 0, st>>>(D, G, NG, x, sm, o); break;
+    case 4: k_scatter<4, I><<<g, kThreads, 0, st>>>(D, G, NG, x, sm, o); break;
+    case 5: k_scatter<5, I><<<g, kThreads, 0, st>>>(D, G, NG, x, sm, o); break;
+    case 6: k_scatter<6, I><<<g, kThreads, 0, st>>>(D, G, NG, x, sm, o); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
 }
 
 template <typename I>
-cudaError_t gather_bwd_L(const LhDims& D, unsigned g, const uint4* a, const uint4* b,
+cudaError_t gather_bwd_L(const LhDims& D, unsigned g, int G, I NG, const uint4* a, const uint4* b,
                          const uint4* c, const int32_t* sm, uint4* x, uint4* y, uint4* z,
                          cudaStream_t st) {
   switch (D.L) {
-    case 1: k_gather_bwd<1, I><<<g, kThreads, 0, st>>>(D, a, b, c, sm, x, y, z); break;
-    case 2: k_gather_bwd<2, I><<<g, kThreads, 0, st>>>(D, a, b, c, sm, x, y, z); break;
-    case 3: k_gather_bwd<3, I><<<g, kThreads, 0, st>>>(D, a, b, c, sm, x, y, z); break;
-    case 4: k_gather_bwd<4, I><<<g, kThreads, 0, st>>>(D, a, b, c, sm, x, y, z); break;
-    case 5: k_gather_bwd<5, I><<<g, kThreads, 0, st>>>(D, a, b, c, sm, x, y, z); break;
-    case 6: k_gather_bwd<6, I><<<g, kThreads, 0, st>>>(D, a, b, c, sm, x, y, z); break;
+    case 1: k_gather_bwd<1, I><<<g, kThreads, 0, st>>>(D, G, NG, a, b, c, sm, x, y, z); break;
+    case 2: k_gather_bwd<2, I><<<g, kThreads, 0, st>>>(D, G, NG, a, b, c, sm, x, y, z); break;
+    case 3: k_gather_bwd<3, I><<<g, kThreads, 0, st>>>(D, G, NG, a, b, c, sm, x, y, z); break;
+    case 4: k_gather_bwd<4, I><<<g, kThreads, 0, st>>>(D, G, NG, a, b, c, sm, x, y, z); break;
+    case 5: k_gather_bwd<5, I><<<g, kThreads, 0, st>>>(D, G, NG, a, b, c, sm, x, y, z); break;
+    case 6: k_gather_bwd<6, I><<<g, kThreads, 0, st>>>(D, G, NG, a, b, c, sm, x, y, z); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
+}
+
+// G of k_scatter / k_gather_bwd: the largest of 4, 2, 1 that divides p (for
+// L > 1, p^(L-1) divides N, so G divides N too) or, for L = 1, N.
+inline int token_group(const LhDims& D) {
+  const int64_t m = D.L > 1 ? D.p : D.N;
+  return m % 4 == 0 ? 4 : (m % 2 == 0 ? 2 : 1);
 }
 
 }  // namespace
@@ -335,11 +388,13 @@ cudaError_t lh_launch_gather(const LhDims& D, const lh_bf16* q, const lh_bf16* k
 
 cudaError_t lh_launch_scatter(const LhDims& D, const lh_bf16* og, const int32_t* slot_map,
                               lh_bf16* o, cudaStream_t st) {
-  const int64_t n = (int64_t)D.B * D.N * D.H * (D.d >> 3);
+  const int G = token_group(D);
+  const int64_t NG = D.N / G + 1;  // shifted groups: t + 1 runs over 1..N
+  const int64_t n = (int64_t)D.B * NG * D.H * (D.d >> 3);
   const unsigned g = nblocks(n);
   const uint4* x = (const uint4*)og;
-  if (n < kIdx32) return scatter_L<uint32_t>(D, g, x, slot_map, (uint4*)o, st);
-  return scatter_L<uint64_t>(D, g, x, slot_map, (uint4*)o, st);
+  if (n < kIdx32) return scatter_L<uint32_t>(D, g, G, (uint32_t)NG, x, slot_map, (uint4*)o, st);
+  return scatter_L<uint64_t>(D, g, G, (uint64_t)NG, x, slot_map, (uint4*)o, st);
 }
 
 size_t lh_scatter_atomic_ws_bytes(const LhDims& D) {
@@ -387,10 +442,13 @@ cudaError_t lh_launch_attn_delta(int BH, int64_t S, int d, const lh_bf16* og,
 cudaError_t lh_launch_gather_bwd(const LhDims& D, const lh_bf16* dqg, const lh_bf16* dkg,
                                  const lh_bf16* dvg, const int32_t* slot_map, lh_bf16* dq,
                                  lh_bf16* dk, lh_bf16* dv, cudaStream_t st) {
-  const int64_t n = (int64_t)D.B * D.N * D.H * (D.d >> 3);
+  const int G = token_group(D);
+  const int64_t NG = D.N / G;
+  const int64_t n = (int64_t)D.B * NG * D.H * (D.d >> 3);
   const unsigned g = nblocks(n);
   const uint4 *a = (const uint4*)dqg, *b = (const uint4*)dkg, *c = (const uint4*)dvg;
   uint4 *x = (uint4*)dq, *y = (uint4*)dk, *z = (uint4*)dv;
-  if (n < kIdx32) return gather_bwd_L<uint32_t>(D, g, a, b, c, slot_map, x, y, z, st);
-  return gather_bwd_L<uint64_t>(D, g, a, b, c, slot_map, x, y, z, st);
+  if (n < kIdx32)
+    return gather_bwd_L<uint32_t>(D, g, G, (uint32_t)NG, a, b, c, slot_map, x, y, z, st);
+  return gather_bwd_L<uint64_t>(D, g, G, (uint64_t)NG, a, b, c, slot_map, x, y, z, st);
 }

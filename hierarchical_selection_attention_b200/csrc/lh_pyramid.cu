@@ -4,21 +4,50 @@
 //
 // One thread owns one 16-byte vector (8 features) of one (token, head) row
 // and walks the W = p^(L-1) tokens of one coarsest window.  Consecutive
-// threads own consecutive vectors of a token row, so every warp-wide load is
-// 512 contiguous bytes.  Per token the thread:
+// threads own consecutive vectors of a token row, so every warp-wide copy is
+// 512 contiguous bytes.  The thread streams its vectors of Q, K and V through
+// a private ring of kDepth token slots in shared memory (cp.async, 16 bytes
+// per copy): up to kDepth - 1 tokens are in flight while it works on the
+// current one, and as each thread reads only what it copied itself, no block
+// barrier is needed.  Per token the thread:
 //   * adds its 8 values of Q, K and V into fp32 running sums, one per level
 //     l >= 1, and writes level l's mean (rounded once to bf16) after every p^l
 //     tokens;
 //   * sums its 8 squares of Q and of K in fp64; the d/8 lanes of the row then
-//     combine their partial sums with xor shuffles, and the fp64 square root,
-//     rounded once to fp32, is the level-0 score (bf16 squares are exact in
+//     combine their partial sums with xor shuffles (bf16 squares are exact in
 //     fp64, so the sum is the exact one whenever the row's magnitudes span
 //     less than about 2^15, and any rounding it does is 2^-53-relative);
-//   * keeps the running max of the level-0 scores per level: a coarse score
-//     is the max of the level-0 scores in its window.
+//   * keeps, per level l >= 1, the running max of those squared norms.
+// A score is the fp64 square root of a squared norm, rounded once to fp32; a
+// coarse score is the max of the level-0 scores in its window, which is the
+// root of the max squared norm, since x -> fp32(sqrt(x)) is monotone, so it
+// takes one root per coarse entry.  Level-0 roots are taken in lane batches:
+// the squared norm of the window's j-th token waits in lane j mod (d/8) until
+// the batch is full, and then every lane of the row takes one root and the
+// batch goes out as one contiguous store.
 #include "lh_common.cuh"
 
 namespace {
+
+constexpr int kDepth = 4;  // token slots in each thread's ring
+
+__device__ __forceinline__ void cp_async16(uint4* dst, const uint4* src) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ float root_score(double sq) {
+  return __double2float_rn(__dsqrt_rn(sq));
+}
 
 template <int L>
 __global__ void __launch_bounds__(256, 2) k_pyramid_score(LhDims D, const uint4* __restrict__ q,
@@ -29,9 +58,10 @@ __global__ void __launch_bounds__(256, 2) k_pyramid_score(LhDims D, const uint4*
                                                        uint4* __restrict__ v_lv,
                                                        float* __restrict__ qk,
                                                        float* __restrict__ kq) {
-  const int V = D.d >> 3;                  // vectors per row
+  extern __shared__ uint4 ring[];          // [kDepth][3][blockDim.x]
+  const int V = D.d >> 3;                  // vectors per row (8 or 16)
   const int HV = D.H * V;                  // vectors per token
-  const int64_t W = D.lvl_span[L - 1];     // tokens per coarsest window
+  const int W = (int)D.lvl_span[L - 1];    // tokens per coarsest window
   const int64_t n_win = D.N / W;
   const int64_t item = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t total = (int64_t)D.B * n_win * HV;
@@ -50,26 +80,63 @@ __global__ void __launch_bounds__(256, 2) k_pyramid_score(LhDims D, const uint4*
   float* qk_row = qk + bh * D.P;
   float* kq_row = kq + bh * D.P;
 
+  const int64_t row0 = ((int64_t)b * D.N + t0) * HV + j;   // vector index of token t0
+  const uint4* gq = q + row0;
+  const uint4* gk = k + row0;
+  const uint4* gv = v + row0;
+  const unsigned nt = blockDim.x;
+  uint4* mine = ring + threadIdx.x;
+  auto stage = [&](int t) {  // copy token t's three vectors into slot t mod kDepth
+    if (t < W) {
+      uint4* dst = mine + (t % kDepth) * 3 * nt;
+      const int64_t off = (int64_t)t * HV;
+      cp_async16(dst, gq + off);
+      cp_async16(dst + nt, gk + off);
+      cp_async16(dst + 2 * nt, gv + off);
+    }
+    cp_async_commit();  // one group per token, empty past the window
+  };
+
   float aq[L > 1 ? L - 1 : 1][8], ak[L > 1 ? L - 1 : 1][8], av[L > 1 ? L - 1 : 1][8];
-  float mq[L], mk[L];
-  int left[L];        // tokens still to add before level l's entry is complete
-  int64_t ent[L];     // index of level l's current entry
+  double mq[L], mk[L];   // running max squared norms, levels >= 1
+  double pq = 0.0, pk = 0.0;   // level-0 squared norms parked until their batch is rooted
+  int left[L];           // tokens still to add before level l's entry is complete
+  int ent[L];            // index of level l's current entry (P < 2^31)
 #pragma unroll
   for (int l = 0; l < L - 1; ++l)
 #pragma unroll
     for (int e = 0; e < 8; ++e) aq[l][e] = ak[l][e] = av[l][e] = 0.f;
 #pragma unroll
   for (int l = 0; l < L; ++l) {
-    mq[l] = mk[l] = 0.f;
+    mq[l] = mk[l] = 0.0;
     left[l] = (int)D.lvl_span[l];
-    ent[l] = t0 / D.lvl_span[l];
+    ent[l] = (int)(t0 / D.lvl_span[l]);
   }
+  // Token t is complete with squared norms (sq, sk): park them in lane
+  // t mod V, and once the batch is full or the window ends, the batch's lanes
+  // write their roots.
+  auto settle0 = [&](int t, double sq, double sk) {
+    const int pos = t & (V - 1);
+    if (pos == cv) {
+      pq = sq;
+      pk = sk;
+    }
+    if ((pos == V - 1 || t == W - 1) && cv <= pos) {
+      const int64_t e = D.lvl_off[0] + t0 + (t - pos) + cv;
+      qk_row[e] = root_score(pq);
+      kq_row[e] = root_score(pk);
+    }
+  };
 
-  const int64_t row0 = ((int64_t)b * D.N + t0) * HV + j;   // vector index of token t0
-#pragma unroll 2
-  for (int t = 0; t < (int)W; ++t) {
-    const int64_t idx = row0 + t * HV;
-    const uint4 uq = __ldg(q + idx), uk = __ldg(k + idx), uv = __ldg(v + idx);
+#pragma unroll
+  for (int s = 0; s < kDepth - 1; ++s) stage(s);
+#pragma unroll 1
+  for (int t = 0; t < W; ++t) {
+    // slot (t - 1) mod kDepth was read and used in the previous iteration
+    stage(t + kDepth - 1);
+    cp_async_wait<kDepth - 1>();   // token t's group has landed
+    const uint4* src = mine + (t % kDepth) * 3 * nt;
+    const uint4 uq = src[0], uk = src[nt], uv = src[2 * nt];
     const uint32_t wq[4] = {uq.x, uq.y, uq.z, uq.w};
     const uint32_t wk[4] = {uk.x, uk.y, uk.z, uk.w};
     const uint32_t wv[4] = {uv.x, uv.y, uv.z, uv.w};
@@ -81,27 +148,28 @@ __global__ void __launch_bounds__(256, 2) k_pyramid_score(LhDims D, const uint4*
       xk[2 * e] = c.x; xk[2 * e + 1] = c.y;
       xv[2 * e] = g.x; xv[2 * e + 1] = g.y;
     }
-    double sq = 0.0, sk = 0.0;
+    // squares summed as a tree (each product is exact in fp64)
+    double sq, sk;
+    {
+      double tq[4], tk[4];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      sq = __fma_rn((double)xq[e], (double)xq[e], sq);
-      sk = __fma_rn((double)xk[e], (double)xk[e], sk);
+      for (int e = 0; e < 4; ++e) {
+        const double a0 = xq[2 * e], a1 = xq[2 * e + 1], c0 = xk[2 * e], c1 = xk[2 * e + 1];
+        tq[e] = __fma_rn(a0, a0, a1 * a1);
+        tk[e] = __fma_rn(c0, c0, c1 * c1);
+      }
+      sq = (tq[0] + tq[1]) + (tq[2] + tq[3]);
+      sk = (tk[0] + tk[1]) + (tk[2] + tk[3]);
     }
     for (int o = V >> 1; o > 0; o >>= 1) {
       sq += __shfl_xor_sync(live, sq, o);
       sk += __shfl_xor_sync(live, sk, o);
     }
-    const float nq = __double2float_rn(__dsqrt_rn(sq));
-    const float nk = __double2float_rn(__dsqrt_rn(sk));
-    const int64_t tok = t0 + t;
-    if (cv == 0) {
-      qk_row[tok] = nq;
-      kq_row[tok] = nk;
-    }
+    settle0(t, sq, sk);
 #pragma unroll
     for (int l = 1; l < L; ++l) {
-      mq[l] = fmaxf(mq[l], nq);
-      mk[l] = fmaxf(mk[l], nk);
+      mq[l] = fmax(mq[l], sq);
+      mk[l] = fmax(mk[l], sk);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         aq[l - 1][e] += xq[e];
@@ -109,7 +177,7 @@ __global__ void __launch_bounds__(256, 2) k_pyramid_score(LhDims D, const uint4*
         av[l - 1][e] += xv[e];
       }
       if (--left[l] == 0) {
-        const int64_t i = ent[l]++;
+        const int i = ent[l]++;
         left[l] = (int)D.lvl_span[l];
         const float fs = (float)D.lvl_span[l];
         // x / p^l; for a power-of-two span the product with the exact
@@ -118,11 +186,11 @@ __global__ void __launch_bounds__(256, 2) k_pyramid_score(LhDims D, const uint4*
         const float inv = 1.f / fs;
         auto mean = [&](float x) { return pow2 ? x * inv : __fdiv_rn(x, fs); };
         uint4 oq, ok, ov;
-        uint32_t* pq = &oq.x; uint32_t* pk = &ok.x; uint32_t* pv = &ov.x;
+        uint32_t* po = &oq.x; uint32_t* pk2 = &ok.x; uint32_t* pv = &ov.x;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          pq[e] = pack_bf16x2(mean(aq[l - 1][2 * e]), mean(aq[l - 1][2 * e + 1]));
-          pk[e] = pack_bf16x2(mean(ak[l - 1][2 * e]), mean(ak[l - 1][2 * e + 1]));
+          po[e] = pack_bf16x2(mean(aq[l - 1][2 * e]), mean(aq[l - 1][2 * e + 1]));
+          pk2[e] = pack_bf16x2(mean(ak[l - 1][2 * e]), mean(ak[l - 1][2 * e + 1]));
           pv[e] = pack_bf16x2(mean(av[l - 1][2 * e]), mean(av[l - 1][2 * e + 1]));
         }
         const int64_t orow = ((int64_t)D.B * D.pool_row[l] + (int64_t)b * D.lvl_size[l] + i) * HV + j;
@@ -132,10 +200,10 @@ __global__ void __launch_bounds__(256, 2) k_pyramid_score(LhDims D, const uint4*
 #pragma unroll
         for (int e = 0; e < 8; ++e) aq[l - 1][e] = ak[l - 1][e] = av[l - 1][e] = 0.f;
         if (cv == 0) {
-          qk_row[D.lvl_off[l] + i] = mq[l];
-          kq_row[D.lvl_off[l] + i] = mk[l];
+          qk_row[D.lvl_off[l] + i] = root_score(mq[l]);
+          kq_row[D.lvl_off[l] + i] = root_score(mk[l]);
         }
-        mq[l] = mk[l] = 0.f;
+        mq[l] = mk[l] = 0.0;
       }
     }
   }
@@ -148,8 +216,12 @@ cudaError_t launch_L(const LhDims& D, const lh_bf16* q, const lh_bf16* k, const 
   const int64_t HV = (int64_t)D.H * (D.d >> 3);
   const int64_t total = (int64_t)D.B * (D.N / D.lvl_span[L - 1]) * HV;
   const int threads = 256;
+  const size_t smem = (size_t)kDepth * 3 * threads * sizeof(uint4);   // 48 KB
+  cudaError_t e = cudaFuncSetAttribute(k_pyramid_score<L>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
   const int64_t blocks = (total + threads - 1) / threads;
-  k_pyramid_score<L><<<(unsigned)blocks, threads, 0, st>>>(
+  k_pyramid_score<L><<<(unsigned)blocks, threads, smem, st>>>(
       D, reinterpret_cast<const uint4*>(q), reinterpret_cast<const uint4*>(k),
       reinterpret_cast<const uint4*>(v), reinterpret_cast<uint4*>(q_lv),
       reinterpret_cast<uint4*>(k_lv), reinterpret_cast<uint4*>(v_lv), qk, kq);
