@@ -89,7 +89,7 @@ constexpr int kMaxG = 4;
 // issued before any row load, and all row loads before the sums; each row is
 // summed in ascending level order.
 template <int L, typename I>
-__global__ void __launch_bounds__(kThreads) k_scatter(LhDims D, int G, I NG,
+__global__ void __launch_bounds__(kThreads, 6) k_scatter(LhDims D, int G, I NG,
                                                       const uint4* __restrict__ og,
                                                       const int32_t* __restrict__ slot_map,
                                                       uint4* __restrict__ o) {
