@@ -40,7 +40,11 @@ design notes of the repository):
   entries ending on the same token are ordered child before parent
   (ascending level);
 * softmax scale 1/sqrt(d); positions no entry reaches get 0;
-* selection is per (batch, head).
+* selection is per (batch, head);
+* the stratified selection (mode 2) cuts the finer-level stream, in flat
+  index order, into n_sel / m near-equal contiguous chunks and keeps the top
+  m of each; the pages leave the chunk size to an appendix they do not
+  include, so m is a parameter.
 
 ``parity=True`` rounds values to bf16 where the library stores them (pooled
 entries, the gathered output, its gradient and the gathered gradients) and
@@ -91,7 +95,7 @@ def subseq_len(N: int, L: int, p: int, k: int) -> int:
     return N // p ** (L - 1) + n_select(L, p, k)
 
 
-def check_config(N: int, L: int, p: int, k: int, mode: int = 0) -> None:
+def check_config(N: int, L: int, p: int, k: int, mode: int = 0, chunk: int = 0) -> None:
     if p < 2 or L < 1 or N < 1 or k < 0:
         raise ValueError("need p >= 2, L >= 1, N >= 1, k >= 0")
     if N % p ** (L - 1):
@@ -100,6 +104,10 @@ def check_config(N: int, L: int, p: int, k: int, mode: int = 0) -> None:
         raise ValueError("(L-1) p k exceeds the number of finer-level entries")
     if mode == 1 and L > 1 and p * k > N // p ** (L - 2):
         raise ValueError("per-level quota: p k exceeds the entries of the coarsest finer level")
+    if mode == 2 and (chunk < 1 or n_select(L, p, k) % chunk):
+        raise ValueError("stratified selection: the chunk quota must be >= 1 and divide (L-1) p k")
+    if mode not in (0, 1, 2):
+        raise ValueError("select mode must be 0 (joint), 1 (per-level quota) or 2 (stratified)")
 
 
 def entry_level_index(f: np.ndarray, N: int, L: int, p: int):
@@ -180,7 +188,7 @@ def scores(qh: np.ndarray, kh: np.ndarray, L: int, p: int):
 
 
 def select(qk: np.ndarray, kq: np.ndarray, N: int, L: int, p: int, k: int,
-           mode: int = 0) -> np.ndarray:
+           mode: int = 0, chunk: int = 0) -> np.ndarray:
     """Selection flags over all flat pyramid indices of one head.
 
     mode 0 (joint, Sec. 3.4): the QK and KQ streams of the finer levels are
@@ -191,7 +199,14 @@ def select(qk: np.ndarray, kq: np.ndarray, N: int, L: int, p: int, k: int,
     the L-1 finer levels contributes p k entries): the same walk, but over
     one finer level at a time, taking p k distinct entries from each.
 
-    Level L-1 is kept whole in both modes.
+    mode 2 (stratified, the implementation note of Sec. 3: the score stream
+    is partitioned into chunks and each chunk keeps its own top m): the
+    finer-level entries, in flat-index order, are cut into n_sel / m
+    contiguous chunks, chunk s covering [floor(s C / n), floor((s+1) C / n))
+    for C candidates and n chunks; each chunk takes m = ``chunk`` distinct
+    entries by the same walk.
+
+    Level L-1 is kept whole in every mode.
     """
     C = n_candidates(N, L, p)
     flags = np.zeros(total_entries(N, L, p), dtype=bool)
@@ -200,8 +215,13 @@ def select(qk: np.ndarray, kq: np.ndarray, N: int, L: int, p: int, k: int,
     elif mode == 1:
         offs = level_offsets(N, L, p)
         ranges = [(offs[l], offs[l] + N // p**l, p * k) for l in range(L - 1)]
+    elif mode == 2:
+        if chunk < 1 or n_select(L, p, k) % chunk:
+            raise ValueError("stratified selection: the chunk quota must be >= 1 and divide (L-1) p k")
+        n = n_select(L, p, k) // chunk
+        ranges = [(s * C // n, (s + 1) * C // n, chunk) for s in range(n)]
     else:
-        raise ValueError("select mode must be 0 (joint) or 1 (per-level quota)")
+        raise ValueError("select mode must be 0 (joint), 1 (per-level quota) or 2 (stratified)")
     for lo, hi, take in ranges:
         f = np.arange(lo, hi, dtype=np.int64)
         stream_f = np.concatenate([f, f])
@@ -354,17 +374,18 @@ def pyramid_bwd(dxg: np.ndarray, slot_map: np.ndarray, N: int, L: int, p: int) -
 # --------------------------------------------------------------------------
 
 
-def forward_head(qh, kh, vh, L, p, k, scale=None, parity=True, flags=None, select_mode=0):
+def forward_head(qh, kh, vh, L, p, k, scale=None, parity=True, flags=None, select_mode=0,
+                 select_chunk=0):
     """Forward of one (batch, head).  qh, kh, vh: [N, d] fp64.
 
     ``flags`` freezes the selection (used by gradient and causality checks).
     """
     N, d = qh.shape
-    check_config(N, L, p, k, select_mode)
+    check_config(N, L, p, k, select_mode, select_chunk)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     qk, kq = scores(qh, kh, L, p)
     if flags is None:
-        flags = select(qk, kq, N, L, p, k, select_mode)
+        flags = select(qk, kq, N, L, p, k, select_mode, select_chunk)
     sel_idx, slot_map = gather_order(flags, N, L, p)
     rnd = round_bf16 if parity else (lambda a: a)
     pyr = [pyramid(x, L, p) for x in (qh, kh, vh)]
@@ -396,7 +417,7 @@ def _head(x, b, h) -> np.ndarray:
     return np.ascontiguousarray(np.asarray(x[b, :, h, :], dtype=np.float64))
 
 
-def forward(q, k, v, L, p, kk, scale=None, parity=True, select_mode=0):
+def forward(q, k, v, L, p, kk, scale=None, parity=True, select_mode=0, select_chunk=0):
     """Forward over every (b, h).  q, k, v: arrays [B, N, H, d] (any float
     dtype; converted exactly to fp64 per head).  Returns per-head states in a
     dict keyed by (b, h) and the output O [B, N, H, d]."""
@@ -406,7 +427,8 @@ def forward(q, k, v, L, p, kk, scale=None, parity=True, select_mode=0):
     for b in range(B):
         for h in range(H):
             st = forward_head(_head(q, b, h), _head(k, b, h), _head(v, b, h),
-                              L, p, kk, scale, parity, select_mode=select_mode)
+                              L, p, kk, scale, parity, select_mode=select_mode,
+                              select_chunk=select_chunk)
             states[(b, h)] = st
             o[b, :, h, :] = st["o"]
     return o, states
@@ -427,11 +449,11 @@ def backward(states, do):
 # --------------------------------------------------------------------------
 
 
-def select_head(qh, kh, L, p, k, select_mode=0):
+def select_head(qh, kh, L, p, k, select_mode=0, select_chunk=0):
     """Scores, flags, gather order and slot map of one head (no attention)."""
     N = qh.shape[0]
     qk, kq = scores(qh, kh, L, p)
-    flags = select(qk, kq, N, L, p, k, select_mode)
+    flags = select(qk, kq, N, L, p, k, select_mode, select_chunk)
     sel_idx, slot_map = gather_order(flags, N, L, p)
     return dict(qk=qk, kq=kq, flags=flags, sel_idx=sel_idx, slot_map=slot_map)
 

@@ -84,4 +84,6 @@ def test_quota_config_limits():
         lo.check_config(64, 3, 4, 5, mode=1)      # 20 > 16
     lo.check_config(64, 3, 4, 5, mode=0)          # the joint budget 40 <= 80 candidates
     with pytest.raises(ValueError):
-        lo.select(np.zeros(84), np.zeros(84), 64, 3, 4, 1, mode=2)
+        lo.select(np.zeros(84), np.zeros(84), 64, 3, 4, 1, mode=3)   # no such mode
+    with pytest.raises(ValueError):
+        lo.select(np.zeros(84), np.zeros(84), 64, 3, 4, 1, mode=2)   # stratified needs its quota
