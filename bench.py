@@ -37,6 +37,7 @@ from hierarchical_selection_attention_b200.inputs import WORKLOADS, make_dout, m
 METRIC = "Lighthouse layer fwd & fwd+bwd tokens/s at N=512K on 1 B200; per-stage % roofline"
 UNIT = "tokens/s"
 DEFAULT_WORKLOAD = 3          # n512k_l3_p4_k4096
+SELECT_NAMES = {0: "joint top-k", 1: "per-level quota", 2: "stratified"}
 
 
 def peaks():
@@ -176,8 +177,9 @@ def run_ours(args, w, ws, rank, local):
     qh, kh, vh = make_qkv(B, N, H, d, seed=args.workload)
     doh = make_dout(B, N, H, d, seed=args.workload)
     q, kk, v, dout = (t.to(dev) for t in (qh, kh, vh, doh))
-    cfg = L.make_config(B, N, H, d, Lv, p, k)
-    layer = L.LighthouseLayer(B, N, H, d, Lv, p, k, device=dev)
+    sel = dict(select_mode=args.select_mode, select_chunk=args.select_chunk)
+    cfg = L.make_config(B, N, H, d, Lv, p, k, **sel)
+    layer = L.LighthouseLayer(B, N, H, d, Lv, p, k, device=dev, **sel)
     sv = layer.views()
     e = lambda *s, dt=torch.bfloat16: torch.empty(*s, dtype=dt, device=dev)
     fws, _, _ = L.lh_workspace_bytes(cfg)
@@ -343,7 +345,9 @@ def run_ours(args, w, ws, rank, local):
         "config": {"workload": f"{w['name']}: B={B} N={N} H={H} d={d} L={Lv} p={p} k={k} S={S}",
                    "step": "lh_forward + lh_backward stages (fwd+bwd)",
                    "l2": "inputs larger than L2 (3 GiB of Q,K,V per step); no flush",
-                   "parallelism": f"replicas x{ws} (independent layers, no collective)"},
+                   "parallelism": f"replicas x{ws} (independent layers, no collective)",
+                   "selection": SELECT_NAMES[args.select_mode] +
+                   (f", {args.select_chunk} per chunk" if args.select_mode == 2 else "")},
         "fwd_tokens_per_s": ws * B * N / (fwd_ms / 1e3), "fwd_ms": fwd_ms,
         "stages": per_stage, "roofline": roof, "e2e": e2e, "gpu_launches": launches,
         "clocks": clocks,
@@ -567,6 +571,10 @@ def main():
     ap.add_argument("--sweep", action="store_true",
                     help="latency over N = 8K..512K (one JSON line per N) instead of the bench line")
     ap.add_argument("--no-sdpa", action="store_true", help="--sweep without the dense SDPA context")
+    ap.add_argument("--select-mode", type=int, default=0, choices=[0, 1, 2],
+                    help="selection: 0 joint top-k (default), 1 per-level quota, 2 stratified")
+    ap.add_argument("--select-chunk", type=int, default=0,
+                    help="per-chunk quota m of the stratified selection")
     ap.add_argument("--full-layer", action="store_true",
                     help="time the layer with its Q/K/V/output projections (one JSON line)")
     args = ap.parse_args()

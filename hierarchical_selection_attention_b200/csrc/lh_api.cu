@@ -54,7 +54,11 @@ lh_status check(const lh_config* c) {
   if (P >= (1LL << 31)) return LH_ERR_UNSUPPORTED;
   if (c->d != 64 && c->d != 128) return LH_ERR_UNSUPPORTED;
   if (c->scatter_mode != 0 && c->scatter_mode != 1) return LH_ERR_INVALID_ARGUMENT;
-  if (c->select_mode != 0 && c->select_mode != 1) return LH_ERR_UNSUPPORTED;
+  if (c->select_mode < 0 || c->select_mode > 2) return LH_ERR_UNSUPPORTED;
+  if (c->select_mode == 2 && n_sel > 0) {  // stratified: n_sel / m chunks of the candidates
+    if (c->select_chunk < 1 || n_sel % c->select_chunk) return LH_ERR_INVALID_ARGUMENT;
+    if ((int64_t)c->B * c->H * (n_sel / c->select_chunk) >= (1LL << 31)) return LH_ERR_UNSUPPORTED;
+  }
   if (!(c->scale == c->scale)) return LH_ERR_INVALID_ARGUMENT;
   const int64_t S = c->N / w + n_sel;
   if (S >= (1LL << 31) || (int64_t)c->B * c->H * ((S + 127) / 128) >= (1LL << 31))
@@ -83,7 +87,11 @@ LhDims dims(const lh_config* c) {
   D.n_sel = (int64_t)(D.L - 1) * c->p * c->k;
   D.S = D.lvl_size[D.L - 1] + D.n_sel;
   D.select_mode = c->select_mode;
-  if (c->select_mode == 1 && D.L > 1) {
+  if (c->select_mode == 2 && D.n_sel > 0) {
+    // one segment per chunk; the chunk bounds are computed, not stored
+    D.nseg = (int)(D.n_sel / c->select_chunk);
+    D.seg_need = c->select_chunk;
+  } else if (c->select_mode == 1 && D.L > 1) {
     D.nseg = D.L - 1;
     for (int l = 0; l < D.L - 1; ++l) {
       D.seg_lo[l] = D.lvl_off[l];
@@ -91,6 +99,7 @@ LhDims dims(const lh_config* c) {
     }
     D.seg_need = (int64_t)c->p * c->k;
   } else {
+    D.select_mode = c->select_mode == 1 ? 1 : 0;   // nothing to stratify: one empty segment
     D.nseg = 1;
     D.seg_lo[0] = 0;
     D.seg_len[0] = D.n_cand;
@@ -516,7 +525,8 @@ int32_t lh_forward_launches(const lh_config* cfg) {
   if (check(cfg) != LH_OK) return -1;
   const LhDims D = dims(cfg);
   // kernels only (the memsets of the scratch are copy-engine work, not counted)
-  const int select = D.n_cand > 0 ? 12 + 3 : 1 + 3;  // hist/find pairs + order count/scan/emit
+  // hist/find pairs (one fused chunk kernel when stratified) + order count/scan/emit
+  const int select = D.select_mode == 2 ? 1 + 3 : (D.n_cand > 0 ? 12 + 3 : 1 + 3);
   const int scatter = cfg->scatter_mode == 1 ? 2 : 1;
   return 1 + select + 1 + 1 + scatter;
 }

@@ -24,7 +24,10 @@ struct LhDims {
   int64_t pool_row[LH_MAX_LEVELS];   // first pooled row of level l (l >= 1), per batch row
   int64_t pooled_rows;               // sum_{l>=1} N / p^l
   // Selection segments: select_mode 0 has one (all finer entries, n_sel to
-  // take), select_mode 1 one per finer level (p k to take from each).
+  // take), select_mode 1 one per finer level (p k to take from each),
+  // select_mode 2 one per chunk (nseg chunks of the n_cand candidates, chunk
+  // s = [floor(s n_cand / nseg), floor((s+1) n_cand / nseg)), seg_need each;
+  // seg_lo / seg_len are not used).
   int select_mode;
   int nseg;
   int64_t seg_lo[LH_MAX_LEVELS];     // first flat index of segment s

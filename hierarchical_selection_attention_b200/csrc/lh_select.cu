@@ -19,7 +19,11 @@
 // Selection modes.  Mode 0 runs that selection once over all finer entries
 // (n_sel to take); mode 1, the per-level quota, runs it once per finer level
 // (p k to take from each, Eq. 8 read as an exact per-level count).  Each run
-// is a "segment" with its own histograms, state and threshold.
+// is a "segment" with its own histograms, state and threshold.  Mode 2, the
+// stratified selection, cuts the candidates into n_sel / m contiguous chunks
+// and keeps the top m of each; a chunk is small (about m C / n_sel keys), so
+// one block runs all of its radix passes with the histogram in shared memory
+// and keeps only the final threshold.
 //
 // Order.  Entries are sorted by the last base token they summarise,
 // e = (i+1) p^l - 1, and by level.  Walking the base tokens t in order and,
@@ -155,11 +159,97 @@ __global__ void __launch_bounds__(256) k_sel_find(LhDims D, const unsigned* __re
   }
 }
 
+// Stratified selection: one block of 256 threads per (b, h) and chunk finds
+// the chunk's m-th largest key by the same 11-bit radix passes, reading the
+// chunk's keys once per pass (they stay in L1/L2) and counting digits in
+// shared memory; it stops as soon as every key left in the chosen digit is
+// needed.  state[bs].prefix is then the threshold: selected(f) <=> key(f) >=
+// prefix, and exactly m keys of the chunk pass it (keys are unique).
+__global__ void __launch_bounds__(256) k_sel_chunk(LhDims D, const float* __restrict__ qk,
+                                                   const float* __restrict__ kq,
+                                                   SelState* __restrict__ state) {
+  const int64_t bs = blockIdx.x;                 // (b, h) x chunk
+  const int64_t bh = bs / D.nseg;
+  const int64_t s = bs - bh * D.nseg;
+  const int64_t lo = s * D.n_cand / D.nseg;
+  const int64_t hi_f = (s + 1) * D.n_cand / D.nseg;
+  const float* q = qk + bh * D.P;
+  const float* k = kq + bh * D.P;
+  __shared__ unsigned h[kBins];
+  __shared__ SelState sh;
+  typedef cub::BlockScan<long long, 256> Scan;
+  __shared__ typename Scan::TempStorage tmp;
+  SelState st;
+  st.prefix = 0;
+  st.need = D.seg_need;
+  st.done = 0;
+  st.pad = 0;
+  for (int pass = 0; pass < kPasses; ++pass) {
+    for (int i = threadIdx.x; i < kBins; i += blockDim.x) h[i] = 0;
+    __syncthreads();
+    const int shift = c_shift[pass];
+    const int hi = shift + c_width[pass];
+    const unsigned mask = (1u << c_width[pass]) - 1u;
+    for (int64_t f0 = lo; f0 < hi_f; f0 += blockDim.x) {
+      const int64_t f = f0 + threadIdx.x;
+      bool in = f < hi_f;
+      unsigned digit = 0;
+      if (in) {
+        const unsigned long long key = entry_key(q, k, f);
+        in = (hi >= 64) || ((key >> hi) == (st.prefix >> hi));
+        digit = (unsigned)(key >> shift) & mask;
+      }
+      const unsigned act = __ballot_sync(0xffffffffu, in);
+      if (in) {
+        const unsigned peers = __match_any_sync(act, digit);
+        if ((threadIdx.x & 31) == (unsigned)(__ffs(peers) - 1)) atomicAdd(&h[digit], __popc(peers));
+      }
+    }
+    __syncthreads();
+    unsigned c[8];
+    long long mine = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      c[i] = h[kBins - 1 - (threadIdx.x * 8 + i)];
+      mine += c[i];
+    }
+    long long before;
+    Scan(tmp).ExclusiveSum(mine, before);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (before < st.need && st.need <= before + (long long)c[i]) {
+        const unsigned digit = kBins - 1 - (threadIdx.x * 8 + i);
+        SelState o;
+        o.prefix = st.prefix | ((unsigned long long)digit << c_shift[pass]);
+        o.need = st.need - before;
+        o.done = (o.need == (long long)c[i]) ? 1 : 0;
+        o.pad = 0;
+        sh = o;
+      }
+      before += c[i];
+    }
+    __syncthreads();   // sh written by exactly one thread (need <= keys left)
+    st = sh;
+    __syncthreads();   // everyone has read sh and h before the next pass clears h
+    if (st.done) break;
+  }
+  if (threadIdx.x == 0) {
+    if (!st.done) lh_report(D.status, LH_ERR_DEVICE_BOUNDS, 103);
+    state[bs] = st;
+  }
+}
+
 // thr: the (b, h)'s segment states; an entry of level l < L-1 is compared with
-// the threshold of its segment (segment 0 in mode 0, segment l in mode 1).
+// the threshold of its segment: segment 0 in mode 0, segment l in mode 1, and
+// in mode 2 its chunk s, the one with floor(s C / n) <= f < floor((s+1) C / n),
+// i.e. s = floor(((f+1) n - 1) / C).
 __device__ __forceinline__ bool selected_entry(const LhDims& D, const float* q, const float* k,
                                                const SelState* thr, int l, int64_t f) {
-  return (l == D.L - 1) || (entry_key(q, k, f) >= thr[D.nseg > 1 ? l : 0].prefix);
+  if (l == D.L - 1) return true;
+  int64_t seg = 0;
+  if (D.select_mode == 2) seg = ((f + 1) * D.nseg - 1) / D.n_cand;
+  else if (D.nseg > 1) seg = l;
+  return entry_key(q, k, f) >= thr[seg].prefix;
 }
 
 // Number of selected entries that end on token t.
@@ -268,7 +358,7 @@ size_t lh_select_ws_bytes(const LhDims& D) {
   const int64_t BH = (int64_t)D.B * D.H;
   const int64_t BS = BH * D.nseg;
   size_t b = 0;
-  b += (size_t)BS * kPasses * kBins * sizeof(unsigned);
+  if (D.select_mode != 2) b += (size_t)BS * kPasses * kBins * sizeof(unsigned);  // histograms
   b += (size_t)BS * sizeof(SelState);
   b = (b + 255) & ~(size_t)255;
   b += (size_t)BH * order_blocks(D) * sizeof(int);
@@ -280,16 +370,21 @@ cudaError_t lh_launch_select(const LhDims& D, const float* qk, const float* kq,
                              int* launches) {
   const int64_t BH = (int64_t)D.B * D.H;
   const int64_t BS = BH * D.nseg;                 // (b, h) x selection segment
+  const size_t hist_bytes =
+      D.select_mode == 2 ? 0 : (size_t)BS * kPasses * kBins * sizeof(unsigned);
   unsigned* hist = reinterpret_cast<unsigned*>(ws);
-  SelState* state = reinterpret_cast<SelState*>(hist + BS * kPasses * kBins);
-  size_t off = (size_t)BS * kPasses * kBins * sizeof(unsigned) + (size_t)BS * sizeof(SelState);
+  SelState* state = reinterpret_cast<SelState*>(reinterpret_cast<char*>(ws) + hist_bytes);
+  size_t off = hist_bytes + (size_t)BS * sizeof(SelState);
   off = (off + 255) & ~(size_t)255;
   int* blk = reinterpret_cast<int*>(reinterpret_cast<char*>(ws) + off);
   const int nblk = (int)order_blocks(D);
   int n = 0;
-  cudaError_t e = cudaMemsetAsync(hist, 0, (size_t)BS * kPasses * kBins * sizeof(unsigned), st);
-  if (e != cudaSuccess) return e;
-  if (D.n_cand > 0) {
+  if (D.select_mode == 2) {
+    k_sel_chunk<<<(unsigned)BS, 256, 0, st>>>(D, qk, kq, state);
+    n += 1;
+  } else if (D.n_cand > 0) {
+    cudaError_t e = cudaMemsetAsync(hist, 0, hist_bytes, st);
+    if (e != cudaSuccess) return e;
     // ~8 candidates per thread per block keeps every SM busy on one head too
     int64_t per = (D.seg_len[0] + 148 * 4 - 1) / (148 * 4);   // segment 0 is the largest
     per = per < 2048 ? 2048 : per;
@@ -300,7 +395,7 @@ cudaError_t lh_launch_select(const LhDims& D, const float* qk, const float* kq,
       n += 2;
     }
   } else {
-    k_sel_find<<<(unsigned)BS, 256, 0, st>>>(D, hist, state, 0);
+    k_sel_find<<<(unsigned)BS, 256, 0, st>>>(D, hist, state, 0);   // reads no histogram
     n += 1;
   }
   k_order_count<<<dim3(nblk, (unsigned)BH), kOrderThreads, 0, st>>>(D, qk, kq, state, blk, nblk);

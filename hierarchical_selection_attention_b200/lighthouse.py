@@ -34,7 +34,8 @@ class lh_config(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int64), ("N", ctypes.c_int64), ("H", ctypes.c_int64),
                 ("d", ctypes.c_int64), ("L", ctypes.c_int64), ("p", ctypes.c_int64),
                 ("k", ctypes.c_int64), ("scale", ctypes.c_float),
-                ("scatter_mode", ctypes.c_int32), ("select_mode", ctypes.c_int32)]
+                ("scatter_mode", ctypes.c_int32), ("select_mode", ctypes.c_int32),
+                ("select_chunk", ctypes.c_int64)]
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}
@@ -97,8 +98,8 @@ EXPORTED = ("lh_config_check", "lh_subseq_len", "lh_total_entries", "lh_pooled_r
 
 
 def make_config(B, N, H, d, L, p, k, scale: float = 0.0, scatter_mode: int = 0,
-                select_mode: int = 0) -> lh_config:
-    return lh_config(B, N, H, d, L, p, k, scale, scatter_mode, select_mode)
+                select_mode: int = 0, select_chunk: int = 0) -> lh_config:
+    return lh_config(B, N, H, d, L, p, k, scale, scatter_mode, select_mode, select_chunk)
 
 
 def _ck(code: int, where: str):
@@ -324,8 +325,9 @@ class LighthouseLayer:
     """
 
     def __init__(self, B, N, H, d, L, p, k, scale: float = 0.0, scatter_mode: int = 0,
-                 device="cuda", select_mode: int = 0):
-        self.cfg = make_config(B, N, H, d, L, p, k, scale, scatter_mode, select_mode)
+                 device="cuda", select_mode: int = 0, select_chunk: int = 0):
+        self.cfg = make_config(B, N, H, d, L, p, k, scale, scatter_mode, select_mode,
+                               select_chunk)
         _ck(lh_config_check(self.cfg), "lh_config_check")
         fwd, bwd, saved = lh_workspace_bytes(self.cfg)
         self.device = torch.device(device)
@@ -362,9 +364,9 @@ class LighthouseProjectedLayer:
     """
 
     def __init__(self, B, N, H, d, Dm, L, p, k, scale: float = 0.0, device="cuda",
-                 select_mode: int = 0):
+                 select_mode: int = 0, select_chunk: int = 0):
         self.core = LighthouseLayer(B, N, H, d, L, p, k, scale, device=device,
-                                    select_mode=select_mode)
+                                    select_mode=select_mode, select_chunk=select_chunk)
         self.shape = (B, N, H, d, Dm)
         dev = self.core.device
         e = lambda *s: torch.empty(*s, dtype=BF16, device=dev)

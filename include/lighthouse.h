@@ -68,13 +68,22 @@ typedef enum {
  * select_mode: 0 = one joint top-k over all finer levels (Sec. 3.4);
  *   1 = per-level quota: each of the L-1 finer levels contributes exactly
  *   p k entries (the Eq. 8 accounting read literally), chosen within the
- *   level by the same key order; needs p k <= N / p^(L-2).  S is the same in
- *   both modes.  Other values: LH_ERR_UNSUPPORTED. */
+ *   level by the same key order; needs p k <= N / p^(L-2);
+ *   2 = stratified (the chunked top-k of the implementation note in Sec. 3):
+ *   the finer-level entries, in flat-index order, are cut into
+ *   n = (L-1) p k / select_chunk contiguous chunks, chunk s covering
+ *   [floor(s C / n), floor((s+1) C / n)) of the C candidates, and each chunk
+ *   keeps its top select_chunk entries by the same key order; select_chunk
+ *   must be >= 1 and divide (L-1) p k (else LH_ERR_INVALID_ARGUMENT), and
+ *   B H n must be below 2^31 (else LH_ERR_UNSUPPORTED).
+ *   S is the same in every mode.  Other values: LH_ERR_UNSUPPORTED.
+ * select_chunk: the per-chunk quota m of select_mode 2; ignored otherwise. */
 typedef struct {
   int64_t B, N, H, d, L, p, k;
   float scale;
   int32_t scatter_mode;
   int32_t select_mode;
+  int64_t select_chunk;
 } lh_config;
 
 /* Returns LH_OK when the config is valid and supported: B, N, H >= 1,

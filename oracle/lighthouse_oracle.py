@@ -104,7 +104,7 @@ def check_config(N: int, L: int, p: int, k: int, mode: int = 0, chunk: int = 0) 
         raise ValueError("(L-1) p k exceeds the number of finer-level entries")
     if mode == 1 and L > 1 and p * k > N // p ** (L - 2):
         raise ValueError("per-level quota: p k exceeds the entries of the coarsest finer level")
-    if mode == 2 and (chunk < 1 or n_select(L, p, k) % chunk):
+    if mode == 2 and n_select(L, p, k) and (chunk < 1 or n_select(L, p, k) % chunk):
         raise ValueError("stratified selection: the chunk quota must be >= 1 and divide (L-1) p k")
     if mode not in (0, 1, 2):
         raise ValueError("select mode must be 0 (joint), 1 (per-level quota) or 2 (stratified)")
@@ -216,9 +216,10 @@ def select(qk: np.ndarray, kq: np.ndarray, N: int, L: int, p: int, k: int,
         offs = level_offsets(N, L, p)
         ranges = [(offs[l], offs[l] + N // p**l, p * k) for l in range(L - 1)]
     elif mode == 2:
-        if chunk < 1 or n_select(L, p, k) % chunk:
+        n_sel = n_select(L, p, k)
+        if n_sel and (chunk < 1 or n_sel % chunk):
             raise ValueError("stratified selection: the chunk quota must be >= 1 and divide (L-1) p k")
-        n = n_select(L, p, k) // chunk
+        n = n_sel // chunk if n_sel else 0      # nothing to take: no chunks
         ranges = [(s * C // n, (s + 1) * C // n, chunk) for s in range(n)]
     else:
         raise ValueError("select mode must be 0 (joint), 1 (per-level quota) or 2 (stratified)")

@@ -79,20 +79,29 @@ def test_launch_counts(L):
     assert L.lh_forward_launches(L.make_config(1, 100, 2, 64, 3, 4, 1)) == -1
 
 
-@pytest.mark.parametrize("mode,N,L_,p,k,code", [
-    (1, 4096, 3, 4, 64, 0),     # per-level quota: p k = 256 <= N / p = 1024
-    (1, 64, 3, 4, 4, 0),        # p k = 16 == the coarsest finer level
-    (1, 64, 3, 4, 5, 1),        # p k = 20 > 16 (the joint mode accepts it)
-    (0, 64, 3, 4, 5, 0),
-    (2, 4096, 3, 4, 64, 2),     # no stratified mode
-    (1, 640, 1, 4, 0, 0),       # one level: nothing to select in either mode
+@pytest.mark.parametrize("mode,N,L_,p,k,chunk,code", [
+    (1, 4096, 3, 4, 64, 0, 0),     # per-level quota: p k = 256 <= N / p = 1024
+    (1, 64, 3, 4, 4, 0, 0),        # p k = 16 == the coarsest finer level
+    (1, 64, 3, 4, 5, 0, 1),        # p k = 20 > 16 (the joint mode accepts it)
+    (0, 64, 3, 4, 5, 0, 0),
+    (2, 4096, 3, 4, 64, 64, 0),    # stratified: 512 / 64 = 8 chunks
+    (2, 4096, 3, 4, 64, 512, 0),   # one chunk (the joint selection)
+    (2, 4096, 3, 4, 64, 0, 1),     # no chunk quota
+    (2, 4096, 3, 4, 64, 48, 1),    # 48 does not divide 512
+    (2, 4096, 3, 4, 0, 0, 0),      # nothing to select: no chunks needed
+    (3, 4096, 3, 4, 64, 0, 2),     # no such mode
+    (1, 640, 1, 4, 0, 0, 0),       # one level: nothing to select in any mode
 ])
-def test_select_mode_config(L, mode, N, L_, p, k, code):
-    cfg = L.make_config(1, N, 2, 64, L_, p, k, select_mode=mode)
+def test_select_mode_config(L, mode, N, L_, p, k, chunk, code):
+    cfg = L.make_config(1, N, 2, 64, L_, p, k, select_mode=mode, select_chunk=chunk)
     assert L.lh_config_check(cfg) == code
     if code == 0:
         # S does not depend on the selection mode
         assert L.lh_subseq_len(cfg) == lo.subseq_len(N, L_, p, k)
+        lo.check_config(N, L_, p, k, mode, chunk)   # the oracle accepts it too
+    elif code == 1:
+        with pytest.raises(ValueError):
+            lo.check_config(N, L_, p, k, mode, chunk)
 
 
 def test_quota_mode_needs_a_larger_selection_workspace(L):
@@ -100,6 +109,17 @@ def test_quota_mode_needs_a_larger_selection_workspace(L):
     f0, _, _ = L.lh_workspace_bytes(L.make_config(1, 4096, 2, 64, 3, 4, 64))
     f1, _, _ = L.lh_workspace_bytes(L.make_config(1, 4096, 2, 64, 3, 4, 64, select_mode=1))
     assert f1 > f0
+
+
+def test_stratified_mode_needs_no_histograms(L):
+    # a chunk keeps only its threshold state: no per-pass global histograms
+    f0, _, _ = L.lh_workspace_bytes(L.make_config(1, 4096, 2, 64, 3, 4, 64))
+    f2, _, _ = L.lh_workspace_bytes(L.make_config(1, 4096, 2, 64, 3, 4, 64, select_mode=2,
+                                                  select_chunk=64))
+    assert f2 < f0
+    assert L.lh_forward_launches(L.make_config(1, 4096, 2, 64, 3, 4, 64, select_mode=2,
+                                               select_chunk=64)) == \
+        L.lh_forward_launches(L.make_config(1, 4096, 2, 64, 3, 4, 64)) - 11
 
 
 def test_gemm_argument_checks(L):
