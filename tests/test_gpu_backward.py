@@ -23,6 +23,8 @@ CASES = [
     (1, 1000, 2, 64, 2, 2, 50, 3),
     (1, 1024, 2, 128, 4, 2, 20, 4),
     (1, 256, 1, 64, 3, 4, 3, 5),        # S = 40
+    (1, 972, 2, 64, 3, 3, 20, 6),       # p = 3: one token per scatter thread, window 9, S = 228
+    (1, 515, 1, 128, 1, 2, 0, 7),       # L = 1 with odd N: dense causal over 515
 ]
 
 
