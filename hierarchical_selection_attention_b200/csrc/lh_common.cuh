@@ -52,6 +52,24 @@ __device__ __forceinline__ int lh_level_of(const LhDims& D, int64_t f) {
   return l;
 }
 
+// 16-byte asynchronous copy global -> shared (cp.async, L1 bypassed), its
+// commit group and the wait for all but the N most recent groups.  Used where
+// a thread copies into shared-memory slots that only it reads back, so the
+// wait alone orders the copy before the read.
+__device__ __forceinline__ void lh_cp_async16(uint4* dst, const uint4* src) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void lh_cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void lh_cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

@@ -257,12 +257,19 @@ __global__ void __launch_bounds__(kThreads) k_attn_delta(int64_t rows, int V,
 // (unshifted) window holds t is i = floor(t / p^l), the same for the whole
 // group at every l >= 1.  Slot lookups first, then every row load, then the
 // sums, each in ascending level order (two memory round trips per G rows).
+// The level-0 rows of the selected tokens (few: most tokens are reached only
+// through coarser entries) are copied into the thread's own shared-memory
+// slots with cp.async instead of being held in registers, which leaves room
+// for three blocks per SM.
+constexpr size_t kGatherBwdSmem = (size_t)kMaxG * 3 * kThreads * sizeof(uint4);   // 48 KB
+
 template <int L, typename I>
-__global__ void __launch_bounds__(kThreads, L <= 4 ? 2 : 1)
+__global__ void __launch_bounds__(kThreads, L <= 4 ? 3 : 1)
     k_gather_bwd(LhDims D, int G, I NG, const uint4* __restrict__ dqg,
                  const uint4* __restrict__ dkg, const uint4* __restrict__ dvg,
                  const int32_t* __restrict__ slot_map, uint4* __restrict__ dq,
                  uint4* __restrict__ dk, uint4* __restrict__ dv) {
+  extern __shared__ uint4 fine[];   // [kMaxG][3][blockDim.x]
   constexpr int LC = L > 1 ? L - 1 : 1;
   const int V = D.d >> 3;
   const I item = (I)blockIdx.x * blockDim.x + threadIdx.x;
@@ -277,12 +284,24 @@ __global__ void __launch_bounds__(kThreads, L <= 4 ? 2 : 1)
   const int64_t bh = (int64_t)b * D.H + h;
   const int32_t* sm = slot_map + bh * D.P;
   const int64_t base = bh * D.S * V + cv;
+  const unsigned nt = blockDim.x;
+  uint4* mine = fine + threadIdx.x;
   int cslot[LC], fslot[kMaxG];
 #pragma unroll
   for (int l = 1; l < L; ++l) cslot[l - 1] = __ldg(sm + D.lvl_off[l] + t0 / D.lvl_span[l]);
 #pragma unroll
   for (int u = 0; u < kMaxG; ++u) fslot[u] = u < G ? __ldg(sm + D.lvl_off[0] + t0 + u) : -1;
-  uint4 cq[LC], ck[LC], cvv[LC], fq[kMaxG], fk[kMaxG], fv[kMaxG];
+#pragma unroll
+  for (int u = 0; u < kMaxG; ++u) {
+    if (fslot[u] >= 0) {
+      const int64_t s = base + (int64_t)fslot[u] * V;
+      lh_cp_async16(mine + (u * 3 + 0) * nt, dqg + s);
+      lh_cp_async16(mine + (u * 3 + 1) * nt, dkg + s);
+      lh_cp_async16(mine + (u * 3 + 2) * nt, dvg + s);
+    }
+  }
+  lh_cp_async_commit();
+  uint4 cq[LC], ck[LC], cvv[LC];
 #pragma unroll
   for (int l = 1; l < L; ++l) {
     if (cslot[l - 1] >= 0) {
@@ -292,24 +311,16 @@ __global__ void __launch_bounds__(kThreads, L <= 4 ? 2 : 1)
       cvv[l - 1] = __ldg(dvg + s);
     }
   }
-#pragma unroll
-  for (int u = 0; u < kMaxG; ++u) {
-    if (fslot[u] >= 0) {
-      const int64_t s = base + (int64_t)fslot[u] * V;
-      fq[u] = __ldg(dqg + s);
-      fk[u] = __ldg(dkg + s);
-      fv[u] = __ldg(dvg + s);
-    }
-  }
+  lh_cp_async_wait<0>();
 #pragma unroll
   for (int u = 0; u < kMaxG; ++u) {
     if (u >= G) continue;
     float aq[8] = {0, 0, 0, 0, 0, 0, 0, 0}, ak[8] = {0, 0, 0, 0, 0, 0, 0, 0},
           av[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (fslot[u] >= 0) {
-      acc8(aq, fq[u]);
-      acc8(ak, fk[u]);
-      acc8(av, fv[u]);
+      acc8(aq, mine[(u * 3 + 0) * nt]);
+      acc8(ak, mine[(u * 3 + 1) * nt]);
+      acc8(av, mine[(u * 3 + 2) * nt]);
     }
 #pragma unroll
     for (int l = 1; l < L; ++l) {
@@ -350,12 +361,12 @@ cudaError_t gather_bwd_L(const LhDims& D, unsigned g, int G, I NG, const uint4* 
                          const uint4* c, const int32_t* sm, uint4* x, uint4* y, uint4* z,
                          cudaStream_t st) {
   switch (D.L) {
-    case 1: k_gather_bwd<1, I><<<g, kThreads, 0, st>>>(D, G, NG, a, b, c, sm, x, y, z); break;
-    case 2: k_gather_bwd<2, I><<<g, kThreads, 0, st>>>(D, G, NG, a, b, c, sm, x, y, z); break;
-    case 3: k_gather_bwd<3, I><<<g, kThreads, 0, st>>>(D, G, NG, a, b, c, sm, x, y, z); break;
-    case 4: k_gather_bwd<4, I><<<g, kThreads, 0, st>>>(D, G, NG, a, b, c, sm, x, y, z); break;
-    case 5: k_gather_bwd<5, I><<<g, kThreads, 0, st>>>(D, G, NG, a, b, c, sm, x, y, z); break;
-    case 6: k_gather_bwd<6, I><<<g, kThreads, 0, st>>>(D, G, NG, a, b, c, sm, x, y, z); break;
+    case 1: k_gather_bwd<1, I><<<g, kThreads, kGatherBwdSmem, st>>>(D, G, NG, a, b, c, sm, x, y, z); break;
+    case 2: k_gather_bwd<2, I><<<g, kThreads, kGatherBwdSmem, st>>>(D, G, NG, a, b, c, sm, x, y, z); break;
+    case 3: k_gather_bwd<3, I><<<g, kThreads, kGatherBwdSmem, st>>>(D, G, NG, a, b, c, sm, x, y, z); break;
+    case 4: k_gather_bwd<4, I><<<g, kThreads, kGatherBwdSmem, st>>>(D, G, NG, a, b, c, sm, x, y, z); break;
+    case 5: k_gather_bwd<5, I><<<g, kThreads, kGatherBwdSmem, st>>>(D, G, NG, a, b, c, sm, x, y, z); break;
+    case 6: k_gather_bwd<6, I><<<g, kThreads, kGatherBwdSmem, st>>>(D, G, NG, a, b, c, sm, x, y, z); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

@@ -34,20 +34,6 @@ namespace {
 
 constexpr int kDepth = 4;  // token slots in each thread's ring
 
-__device__ __forceinline__ void cp_async16(uint4* dst, const uint4* src) {
-  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
-}
-
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 __device__ __forceinline__ float root_score(double sq) {
   return __double2float_rn(__dsqrt_rn(sq));
 }
@@ -95,11 +81,11 @@ __global__ void __launch_bounds__(256, 2) k_pyramid_score(LhDims D, const uint4*
     if (t < W) {
       uint4* dst = mine + (t % kDepth) * 3 * nt;
       const int64_t off = (int64_t)t * HV;
-      cp_async16(dst, gq + off);
-      cp_async16(dst + nt, gk + off);
-      cp_async16(dst + 2 * nt, gv + off);
+      lh_cp_async16(dst, gq + off);
+      lh_cp_async16(dst + nt, gk + off);
+      lh_cp_async16(dst + 2 * nt, gv + off);
     }
-    cp_async_commit();  // one group per token, empty past the window
+    lh_cp_async_commit();  // one group per token, empty past the window
   };
 
   // Level 1 sums in registers: a1[m][e], m = Q, K, V.  Levels l >= 2 keep
@@ -182,7 +168,7 @@ __global__ void __launch_bounds__(256, 2) k_pyramid_score(LhDims D, const uint4*
   for (int t = 0; t < W; ++t) {
     // slot (t - 1) mod kDepth was read and used in the previous iteration
     stage(t + kDepth - 1);
-    cp_async_wait<kDepth - 1>();   // token t's group has landed
+    lh_cp_async_wait<kDepth - 1>();   // token t's group has landed
     const uint4* src = mine + (t % kDepth) * 3 * nt;
     const uint4 u[3] = {src[0], src[nt], src[2 * nt]};
     float x[3][8];
