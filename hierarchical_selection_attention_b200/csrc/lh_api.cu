@@ -456,6 +456,12 @@ lh_status lh_gemm(int64_t M, int64_t N, int32_t npairs, const lh_gemm_operand* o
                            (cudaStream_t)stream, nullptr));
 }
 
+lh_status lh_check_wait_timeout(void* stream) {
+  int* p = status_ptr();
+  if (!p) return LH_ERR_CUDA;
+  return cu(lh_launch_wait_timeout_check(p, LH_WAIT_TIMEOUT_CHECK_DETAIL, (cudaStream_t)stream));
+}
+
 lh_status lh_get_device_status(void* stream, int32_t* detail) {
   int* p = status_ptr();
   if (!p) return LH_ERR_CUDA;

@@ -119,6 +119,9 @@ cudaError_t lh_launch_attn_bwd(int BH, int64_t S, int d, float scale, const lh_b
                                lh_bf16* dkg, lh_bf16* dvg, int* status, cudaStream_t st,
                                int which);
 
+// One warp waiting on an mbarrier nothing completes (lh_selftest.cu).
+cudaError_t lh_launch_wait_timeout_check(int* status, int where, cudaStream_t st);
+
 // Plain GEMM (lh_gemm.cu).
 size_t lh_gemm_partial_bytes(int64_t M, int64_t N, int splits);
 cudaError_t lh_launch_gemm(int64_t M, int64_t N, int npairs, const lh_gemm_operand* ops, int a_mn,

@@ -19,6 +19,8 @@ LIB_PATH = os.path.join(_HERE, "liblighthouse.so")
 
 LH_OK = 0
 LH_ERR_INVALID_ARGUMENT = 1
+LH_ERR_DEVICE_TIMEOUT = 5
+LH_WAIT_TIMEOUT_CHECK_DETAIL = 900   # detail code of lh_check_wait_timeout
 _STATUS = {0: "LH_OK", 1: "LH_ERR_INVALID_ARGUMENT", 2: "LH_ERR_UNSUPPORTED",
            3: "LH_ERR_WORKSPACE", 4: "LH_ERR_CUDA", 5: "LH_ERR_DEVICE_TIMEOUT",
            6: "LH_ERR_DEVICE_BOUNDS"}
@@ -74,6 +76,7 @@ def _load():
         "lh_gather_bwd": (I32, [C, P, P, P, P, P, P, P, P]),
         "lh_forward": (I32, [C, P, P, P, P, P, SZ, P, SZ, P]),
         "lh_backward": (I32, [C, P, SZ, P, P, P, P, P, SZ, P]),
+        "lh_check_wait_timeout": (I32, [P]),
         "lh_get_device_status": (I32, [P, ctypes.POINTER(I32)]),
         "lh_status_string": (ctypes.c_char_p, [I32]),
         "lh_forward_launches": (I32, [C]),
@@ -93,7 +96,8 @@ EXPORTED = ("lh_config_check", "lh_subseq_len", "lh_total_entries", "lh_pooled_r
             "lh_workspace_bytes", "lh_saved_offsets", "lh_pyramid", "lh_score_topk",
             "lh_score_topk_noalloc", "lh_score_topk_noalloc_max_bytes", "lh_gather",
             "lh_attn_fwd", "lh_attn_bwd", "lh_attn_bwd_dkdv", "lh_attn_bwd_dq", "lh_scatter", "lh_scatter_bwd", "lh_gather_bwd",
-            "lh_forward", "lh_backward", "lh_get_device_status", "lh_status_string",
+            "lh_forward", "lh_backward", "lh_check_wait_timeout", "lh_get_device_status",
+            "lh_status_string",
             "lh_forward_launches", "lh_backward_launches", "lh_gemm_ws_bytes", "lh_gemm")
 
 
@@ -261,6 +265,14 @@ def lh_get_device_status(stream=None):
     detail = ctypes.c_int32(0)
     code = _lib.lh_get_device_status(_stream(stream), ctypes.byref(detail))
     return code, detail.value
+
+
+def lh_check_wait_timeout(stream=None):
+    """Enqueue the bounded-wait check: one warp waits on an mbarrier nothing
+    completes until the wait gives up (about 2 s) and records
+    LH_ERR_DEVICE_TIMEOUT (detail LH_WAIT_TIMEOUT_CHECK_DETAIL); read it with
+    lh_get_device_status."""
+    _ck(_lib.lh_check_wait_timeout(_stream(stream)), "lh_check_wait_timeout")
 
 
 def check_device_status(stream=None):

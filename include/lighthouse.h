@@ -279,6 +279,17 @@ lh_status lh_gemm(int64_t M, int64_t N, int32_t npairs, const lh_gemm_operand* o
                   int32_t b_mn, lh_bf16* c, int64_t ldc, int32_t splits, void* ws,
                   size_t ws_bytes, void* stream);
 
+/* Failure-detection check (no fault is involved): enqueues one warp that
+ * waits on an mbarrier nothing arrives at, through the same bounded wait the
+ * attention and GEMM kernels use.  After about 4e9 SM clock cycles (about
+ * 2 s) the wait gives up, records LH_ERR_DEVICE_TIMEOUT with detail
+ * LH_WAIT_TIMEOUT_CHECK_DETAIL in the device status word, and the kernel
+ * returns; the CUDA context stays usable.  Returns LH_OK once the launch is
+ * enqueued (LH_ERR_CUDA if it fails); read the outcome with
+ * lh_get_device_status. */
+#define LH_WAIT_TIMEOUT_CHECK_DETAIL 900
+lh_status lh_check_wait_timeout(void* stream);
+
 /* Synchronises `stream`, returns the first device-side error recorded since
  * the last call (LH_OK if none) and clears it.  *detail (may be NULL)
  * receives a kernel-specific code locating the failure. */
