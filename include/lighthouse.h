@@ -131,8 +131,10 @@ lh_status lh_pyramid(const lh_config* cfg, const lh_bf16* q, const lh_bf16* k,
 /* (ii) joint top-k and the topological order of (iii), Sec. 3.4-3.5.
  * Exactly (L-1) p k entries of levels 0..L-2 are chosen per (b, h) by the
  * key r = max(qk, kq), descending, ties to the lower flat index; all of
- * level L-1 is added.  Entries are ordered by their last base token
- * e = (i+1) p^l - 1, then by level.
+ * level L-1 is added.  select_mode 1 takes p k from each finer level and
+ * select_mode 2 select_chunk from each chunk (see lh_config), by the same
+ * key.  Entries are ordered by their last base token e = (i+1) p^l - 1,
+ * then by level.
  *  sel_idx  out int32 [B, H, S]  flat pyramid index of each slot
  *  slot_map out int32 [B, H, P]  slot of each entry, -1 if not selected
  *  ws       scratch of at least fwd_ws bytes (lh_workspace_bytes)          */
