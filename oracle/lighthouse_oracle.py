@@ -537,3 +537,72 @@ def projected_backward(st, dy):
     dwq, dwk, dwv = (rnd(g.T @ xf) for g in (dq, dk, dv))
     dwo = rnd(dyf.T @ of)
     return dx, dwq, dwk, dwv, dwo
+
+
+# --------------------------------------------------------------------------
+# Context parallelism: the sequence cut into shards (the pages' multi-GPU
+# training note: pyramid, scores and top-k run shard-local, and the gathered
+# sub-sequences go through ring attention)
+# --------------------------------------------------------------------------
+
+
+def cp_forward_head(qh, kh, vh, L, p, k, R, scale=None, parity=True, select_mode=0,
+                    select_chunk=0, flags=None):
+    """Forward of one head with the N tokens cut into R contiguous shards.
+
+    Each shard runs the pyramid, the scores and the selection on its own N/R
+    tokens with the layer's p and k, so its sub-sequence has S(N/R) entries.
+    The shards' sub-sequences, in shard order, are then attended to as one
+    sequence under the causal mask.  That is what a ring over the shards
+    computes: every entry of shard r' < r ends before any entry of shard r,
+    so shard r's rows see all earlier shards' rows, and their own causally.
+    Each shard scatters its own part of the output.  ``flags`` (one array
+    per shard) freezes the selection, as in forward_head.
+    """
+    N, d = qh.shape
+    if R < 1 or N % R:
+        raise ValueError("the shard count must divide N")
+    Ns = N // R
+    check_config(Ns, L, p, k, select_mode, select_chunk)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    rnd = round_bf16 if parity else (lambda a: a)
+    shards = []
+    for r in range(R):
+        sl = slice(r * Ns, (r + 1) * Ns)
+        qk, kq = scores(qh[sl], kh[sl], L, p)
+        fl = select(qk, kq, Ns, L, p, k, select_mode, select_chunk) if flags is None else flags[r]
+        sel_idx, slot_map = gather_order(fl, Ns, L, p)
+        pyr = [pyramid(x[sl], L, p) for x in (qh, kh, vh)]
+        pyr = [[lv[0]] + [rnd(a) for a in lv[1:]] for lv in pyr]
+        qg, kg, vg = (gather_rows(lv, sel_idx, Ns, L, p) for lv in pyr)
+        shards.append(dict(qk=qk, kq=kq, flags=fl, sel_idx=sel_idx, slot_map=slot_map,
+                           qg=qg, kg=kg, vg=vg))
+    qg, kg, vg = (np.concatenate([s[n] for s in shards]) for n in ("qg", "kg", "vg"))
+    og, lse = attention(qg, kg, vg, scale)
+    og = rnd(og)
+    Sr = subseq_len(Ns, L, p, k)
+    o = np.zeros((N, d))
+    for r, s in enumerate(shards):
+        s["og"] = og[r * Sr:(r + 1) * Sr]
+        o[r * Ns:(r + 1) * Ns] = scatter(s["og"], s["slot_map"], Ns, L, p)
+    return dict(shards=shards, qg=qg, kg=kg, vg=vg, og=og, lse=lse, o=o, scale=scale, L=L,
+                p=p, k=k, N=N, R=R, parity=parity)
+
+
+def cp_backward_head(st, doh):
+    """Gradients dQ, dK, dV [N, d] of one sharded head, indices frozen: each
+    shard's scatter adjoint, the attention backward over the concatenated
+    sub-sequences, each shard's gather and pooling adjoint."""
+    N, R, L, p, k = st["N"], st["R"], st["L"], st["p"], st["k"]
+    Ns = N // R
+    Sr = subseq_len(Ns, L, p, k)
+    rnd = round_bf16 if st["parity"] else (lambda a: a)
+    dog = np.concatenate([rnd(scatter_bwd(doh[r * Ns:(r + 1) * Ns], s["sel_idx"], Ns, L, p))
+                          for r, s in enumerate(st["shards"])])
+    dxg = attention_bwd(st["qg"], st["kg"], st["vg"], dog, st["scale"])
+    grads = [np.zeros((N, doh.shape[1])) for _ in range(3)]
+    for r, s in enumerate(st["shards"]):
+        rows = slice(r * Sr, (r + 1) * Sr)
+        for a in range(3):
+            grads[a][r * Ns:(r + 1) * Ns] = pyramid_bwd(rnd(dxg[a][rows]), s["slot_map"], Ns, L, p)
+    return tuple(grads)
