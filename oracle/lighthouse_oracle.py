@@ -44,7 +44,11 @@ design notes of the repository):
 * the stratified selection (mode 2) cuts the finer-level stream, in flat
   index order, into n_sel / m near-equal contiguous chunks and keeps the top
   m of each; the pages leave the chunk size to an appendix they do not
-  include, so m is a parameter.
+  include, so m is a parameter;
+* context parallelism (cp_forward_head) cuts the sequence into R contiguous
+  shards, runs the pyramid, scores and selection per shard with the layer's
+  p and k, and attends over the shards' sub-sequences concatenated in shard
+  order under the plain causal mask (what a ring over the shards computes).
 
 ``parity=True`` rounds values to bf16 where the library stores them (pooled
 entries, the gathered output, its gradient and the gathered gradients) and
