@@ -272,7 +272,10 @@ def gather_rows(levels: list[np.ndarray], sel_idx: np.ndarray, N: int, L: int, p
 
 def attention(qg, kg, vg, scale: float, rows=None, chunk: int = 256):
     """O_m = sum_{m' <= m} softmax_m'(scale q_m . k_m') v_m' and the natural-log
-    LSE of each row, for the requested rows (all by default)."""
+    LSE of each row, for the requested rows (all by default).
+
+    A block of rows only multiplies against the keys up to its last row:
+    later keys are masked for every row of the block (weight exactly 0)."""
     S = qg.shape[0]
     rows = np.arange(S) if rows is None else np.asarray(rows, dtype=np.int64)
     o = np.empty((rows.shape[0], vg.shape[1]))
@@ -280,13 +283,14 @@ def attention(qg, kg, vg, scale: float, rows=None, chunk: int = 256):
     cols = np.arange(S)
     for a in range(0, rows.shape[0], chunk):
         r = rows[a:a + chunk]
-        s = (qg[r] @ kg.T) * scale
-        s[cols[None, :] > r[:, None]] = -np.inf
+        hi = int(r.max()) + 1
+        s = (qg[r] @ kg[:hi].T) * scale
+        s[cols[None, :hi] > r[:, None]] = -np.inf
         mx = s.max(axis=1)
         ex = np.exp(s - mx[:, None])
         z = ex.sum(axis=1)
         lse[a:a + chunk] = mx + np.log(z)
-        o[a:a + chunk] = (ex / z[:, None]) @ vg
+        o[a:a + chunk] = (ex / z[:, None]) @ vg[:hi]
     return o, lse
 
 
@@ -306,16 +310,17 @@ def attention_bwd(qg, kg, vg, dog, scale: float, chunk: int = 256, rows=None):
     rows = np.arange(S) if rows is None else np.asarray(rows, dtype=np.int64)
     for a in range(0, rows.shape[0], chunk):
         r = rows[a:a + chunk]
-        s = (qg[r] @ kg.T) * scale
-        s[cols[None, :] > r[:, None]] = -np.inf
+        hi = int(r.max()) + 1          # keys after the block's last row: P = 0
+        s = (qg[r] @ kg[:hi].T) * scale
+        s[cols[None, :hi] > r[:, None]] = -np.inf
         mx = s.max(axis=1)
         ex = np.exp(s - mx[:, None])
         pr = ex / ex.sum(axis=1)[:, None]
-        dp = dog[r] @ vg.T
+        dp = dog[r] @ vg[:hi].T
         ds = pr * (dp - (pr * dp).sum(axis=1)[:, None])
-        dq[r] = scale * (ds @ kg)
-        dk += scale * (ds.T @ qg[r])
-        dv += pr.T @ dog[r]
+        dq[r] = scale * (ds @ kg[:hi])
+        dk[:hi] += scale * (ds.T @ qg[r])
+        dv[:hi] += pr.T @ dog[r]
     return dq, dk, dv
 
 
