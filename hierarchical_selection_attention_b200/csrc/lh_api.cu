@@ -13,16 +13,14 @@ __device__ int g_status_word[2];  // [code, detail], see lh_get_device_status
 constexpr size_t kAlign = 256;
 inline size_t up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 
+// Device address of the status word on the current device and context.
+// Looked up on every call, not cached: the lookup is a table read in the
+// runtime, is thread-safe, and stays right after a device reset or a new
+// primary context, where a cached address would point at freed memory.
 int* status_ptr() {
-  static int* ptrs[64] = {nullptr};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!ptrs[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
-    ptrs[dev] = static_cast<int*>(p);
-  }
-  return ptrs[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+  return static_cast<int*>(p);
 }
 
 lh_status check(const lh_config* c) {
@@ -63,6 +61,10 @@ lh_status check(const lh_config* c) {
   const int64_t S = c->N / w + n_sel;
   if (S >= (1LL << 31) || (int64_t)c->B * c->H * ((S + 127) / 128) >= (1LL << 31))
     return LH_ERR_UNSUPPORTED;
+  // grids with (b, h) or (b, h) x selection segment in gridDim.y (<= 65535)
+  const int64_t BH = (int64_t)c->B * c->H;
+  const int64_t segs = (c->select_mode == 1 && c->L > 1) ? c->L - 1 : 1;
+  if (BH * segs > 65535) return LH_ERR_UNSUPPORTED;
   return LH_OK;
 }
 
@@ -237,6 +239,18 @@ lh_status lh_saved_offsets(const lh_config* cfg, size_t* offsets) {
   if (!offsets) return LH_ERR_INVALID_ARGUMENT;
   const Saved s = saved_layout(dims(cfg));
   for (int i = 0; i < kSaved; ++i) offsets[i] = s.off[i];
+  return LH_OK;
+}
+
+lh_status lh_bwd_ws_offsets(const lh_config* cfg, size_t* offsets) {
+  LH_TRY(check(cfg));
+  if (!offsets) return LH_ERR_INVALID_ARGUMENT;
+  const BwdWs b = bwd_layout(dims(cfg));
+  offsets[0] = b.delta;
+  offsets[1] = b.dog;
+  offsets[2] = b.dqg;
+  offsets[3] = b.dkg;
+  offsets[4] = b.dvg;
   return LH_OK;
 }
 
@@ -449,10 +463,12 @@ lh_status lh_gemm(int64_t M, int64_t N, int32_t npairs, const lh_gemm_operand* o
   if (splits > total) splits = (int32_t)total;
   if (splits > 1 && (!ws || ws_bytes < lh_gemm_partial_bytes(M, N, splits) || !all_aligned(ws)))
     return LH_ERR_WORKSPACE;
+  int* st = status_ptr();
+  if (!st) return LH_ERR_CUDA;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return cu(lh_launch_gemm(M, N, npairs, ops, a_mn, b_mn, c, ldc, splits, ws, status_ptr(), sms,
+  return cu(lh_launch_gemm(M, N, npairs, ops, a_mn, b_mn, c, ldc, splits, ws, st, sms,
                            (cudaStream_t)stream, nullptr));
 }
 
@@ -493,21 +509,16 @@ const char* lh_status_string(lh_status s) {
 // fixed device array instead; every device that loads the library keeps it
 // until the process exits.  Host code must not hand the array's name to a
 // kernel (on the host it names a stand-in, not device memory): the device
-// address is looked up once per device with cudaGetSymbolAddress and that
-// pointer is what the kernels get.
+// address is looked up with cudaGetSymbolAddress, with the device current,
+// and that pointer is what the kernels get.
 constexpr size_t kNoAllocScratchBytes = (size_t)8 << 20;  // 8 MiB
 static __device__ __align__(256) unsigned char g_topk_scratch[kNoAllocScratchBytes];
 
+// Looked up on every call (see status_ptr): thread-safe, and never stale.
 static void* topk_scratch_ptr() {
-  static void* ptrs[64] = {nullptr};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!ptrs[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_topk_scratch) != cudaSuccess || p == nullptr) return nullptr;
-    ptrs[dev] = p;
-  }
-  return ptrs[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_topk_scratch) != cudaSuccess) return nullptr;
+  return p;
 }
 
 lh_status lh_score_topk_noalloc(const lh_config* cfg, const float* qk, const float* kq,

@@ -62,6 +62,7 @@ def _load():
         "lh_pooled_rows": (I64, [C]),
         "lh_workspace_bytes": (I32, [C, ctypes.POINTER(SZ), ctypes.POINTER(SZ), ctypes.POINTER(SZ)]),
         "lh_saved_offsets": (I32, [C, ctypes.POINTER(SZ)]),
+        "lh_bwd_ws_offsets": (I32, [C, ctypes.POINTER(SZ)]),
         "lh_pyramid": (I32, [C, P, P, P, P, P, P, P, P, P]),
         "lh_score_topk": (I32, [C, P, P, P, P, P, SZ, P]),
         "lh_score_topk_noalloc": (I32, [C, P, P, P, P, P]),
@@ -93,7 +94,7 @@ def _load():
 
 _lib = _load()
 EXPORTED = ("lh_config_check", "lh_subseq_len", "lh_total_entries", "lh_pooled_rows",
-            "lh_workspace_bytes", "lh_saved_offsets", "lh_pyramid", "lh_score_topk",
+            "lh_workspace_bytes", "lh_saved_offsets", "lh_bwd_ws_offsets", "lh_pyramid", "lh_score_topk",
             "lh_score_topk_noalloc", "lh_score_topk_noalloc_max_bytes", "lh_gather",
             "lh_attn_fwd", "lh_attn_bwd", "lh_attn_bwd_dkdv", "lh_attn_bwd_dq", "lh_scatter", "lh_scatter_bwd", "lh_gather_bwd",
             "lh_forward", "lh_backward", "lh_check_wait_timeout", "lh_get_device_status",
@@ -161,6 +162,12 @@ def lh_workspace_bytes(cfg: lh_config):
 def lh_saved_offsets(cfg: lh_config):
     arr = (ctypes.c_size_t * 8)()
     _ck(_lib.lh_saved_offsets(ctypes.byref(cfg), arr), "lh_saved_offsets")
+    return list(arr)
+
+
+def lh_bwd_ws_offsets(cfg: lh_config):
+    arr = (ctypes.c_size_t * 5)()
+    _ck(_lib.lh_bwd_ws_offsets(ctypes.byref(cfg), arr), "lh_bwd_ws_offsets")
     return list(arr)
 
 
@@ -361,6 +368,23 @@ class LighthouseLayer:
 
     def views(self):
         return saved_views(self.cfg, self.saved)
+
+    def bwd_views(self):
+        """Typed views into the backward scratch as lh_backward leaves it:
+        delta, dog, dqg, dkg, dvg (no copies)."""
+        off = lh_bwd_ws_offsets(self.cfg)
+        B, H, d, S = self.cfg.B, self.cfg.H, self.cfg.d, self.S
+
+        def view(i, dtype, shape):
+            n = 1
+            for s in shape:
+                n *= s
+            nbytes = n * torch.tensor([], dtype=dtype).element_size()
+            return self.ws_bwd[off[i]:off[i] + nbytes].view(dtype).view(*shape)
+
+        return dict(delta=view(0, F32, (B, H, S)), dog=view(1, BF16, (B, H, S, d)),
+                    dqg=view(2, BF16, (B, H, S, d)), dkg=view(3, BF16, (B, H, S, d)),
+                    dvg=view(4, BF16, (B, H, S, d)))
 
 
 class LighthouseProjectedLayer:

@@ -88,7 +88,9 @@ typedef struct {
 
 /* Returns LH_OK when the config is valid and supported: B, N, H >= 1,
  * p >= 2, 1 <= L <= 6, p^(L-1) | N, 0 <= (L-1) p k <= sum_{l<L-1} N/p^l,
- * d in {64, 128}, every index fits in int32 per (b, h). */
+ * d in {64, 128}, every index fits in int32 per (b, h), and B H (times L-1
+ * in select_mode 1) <= 65535, the launch-grid limit of the per-head
+ * selection kernels (else LH_ERR_UNSUPPORTED). */
 lh_status lh_config_check(const lh_config* cfg);
 
 /* S = N/p^(L-1) + (L-1) p k (Sec. 3.5, Eq. 8); -1 for an invalid config. */
@@ -112,6 +114,14 @@ lh_status lh_workspace_bytes(const lh_config* cfg, size_t* fwd_ws, size_t* bwd_w
  * [B,H,S]), slot_map (int32 [B,H,P]), qg, kg, vg, og, og_lo (bf16
  * [B,H,S,d]), lse (fp32 [B,H,S]).  `offsets` has room for 8 values. */
 lh_status lh_saved_offsets(const lh_config* cfg, size_t* offsets);
+
+/* Byte offsets inside the backward scratch (bwd_ws) that lh_backward leaves
+ * filled when it returns, in this order: delta (fp32 [B,H,S], D of the
+ * attention backward), dog (bf16 [B,H,S,d], the scatter adjoint), dqg, dkg,
+ * dvg (bf16 [B,H,S,d], the gradients of the gathered sub-sequence).
+ * `offsets` has room for 5 values.  Lets a caller inspect the per-stage
+ * results of the layer backward without a second run. */
+lh_status lh_bwd_ws_offsets(const lh_config* cfg, size_t* offsets);
 
 /* (i) + the level-0/coarse scores of (ii), in one pass over Q, K, V.
  * Sec. 3.3: level l, entry i = mean of base rows i p^l .. (i+1) p^l - 1.
@@ -152,9 +162,13 @@ lh_status lh_score_topk(const lh_config* cfg, const float* qk, const float* kq,
  * loads the library until the process exits.  It allocates nothing and
  * calls no allocating routine.
  *  - Same arguments and results as lh_score_topk, minus ws / ws_bytes.
- *  - Returns LH_ERR_WORKSPACE when the selection scratch of cfg (the fwd_ws
- *    part that lh_score_topk uses) exceeds the array; roughly B*H*50 KB +
- *    B*H*N/256 bytes, so B*H <= 128 fits at N = 2^20.
+ *  - Returns LH_ERR_WORKSPACE, before any launch, when the selection
+ *    scratch of cfg (the part of fwd_ws that lh_score_topk uses) exceeds the
+ *    array.  That scratch is, roughly: select_mode 0, B*H*48 KB of digit
+ *    histograms; select_mode 1, B*H*(L-1)*48 KB; select_mode 2, B*H*n*24
+ *    bytes for its n chunks; plus B*H*N/256 bytes of order counts in every
+ *    mode.  So B*H <= 128 heads fit at N = 2^20 in modes 0 and 2, and
+ *    B*H*(L-1) <= 128 in mode 1.
  *  - The first call on a device looks up the array's device address (once
  *    per device, with that device current); make that first call before any
  *    stream capture.
@@ -187,7 +201,10 @@ lh_status lh_attn_fwd(const lh_config* cfg, const lh_bf16* qg, const lh_bf16* kg
                       const lh_bf16* vg, lh_bf16* og, lh_bf16* og_lo, float* lse,
                       void* stream);
 
-/* Backward of lh_attn_fwd: with P the softmax rows, D = rowsum(dog * O)
+/* Backward of lh_attn_fwd (Sec. 3.2: gradients flow from the loss through
+ * stages (iv) and (iii) into the gathered Q, K, V; the attention is the
+ * masked softmax attention of Sec. 3.5, Eq. 9, so its backward is the
+ * standard one): with P the softmax rows, D = rowsum(dog * O)
  * (O = og + og_lo; og_lo may be NULL), dS = P (dog vg^T - D):
  * dqg = scale dS kg, dkg = scale dS^T qg, dvg = P^T dog.  Deterministic (no
  * floating-point atomics).  Computes D into ws (>= bwd_ws bytes), then runs
@@ -197,15 +214,18 @@ lh_status lh_attn_bwd(const lh_config* cfg, const lh_bf16* qg, const lh_bf16* kg
                       const float* lse, const lh_bf16* dog, lh_bf16* dqg, lh_bf16* dkg,
                       lh_bf16* dvg, void* ws, size_t ws_bytes, void* stream);
 
-/* The dK/dV half of lh_attn_bwd, given delta = D (fp32 [B, H, S], e.g. from
- * lh_scatter_bwd): one CTA per 128 key rows walks the query rows at and
- * after its diagonal.  dkg, dvg out bf16 [B, H, S, d]. */
+/* The dK/dV half of lh_attn_bwd (Sec. 3.2 and 3.5, Eq. 9), given delta = D
+ * (fp32 [B, H, S], e.g. from lh_scatter_bwd): one CTA per 128 key rows walks
+ * the query rows at and after its diagonal.  qg, kg, vg, dog in bf16
+ * [B, H, S, d]; lse in fp32 [B, H, S] from lh_attn_fwd; dkg, dvg out bf16
+ * [B, H, S, d].  Deterministic: each output row is written by one thread. */
 lh_status lh_attn_bwd_dkdv(const lh_config* cfg, const lh_bf16* qg, const lh_bf16* kg,
                            const lh_bf16* vg, const lh_bf16* dog, const float* lse,
                            const float* delta, lh_bf16* dkg, lh_bf16* dvg, void* stream);
 
-/* The dQ half of lh_attn_bwd, given delta: one CTA per 128 query rows walks
- * the key rows up to its diagonal.  dqg out bf16 [B, H, S, d]. */
+/* The dQ half of lh_attn_bwd (Sec. 3.2 and 3.5, Eq. 9), given delta: one
+ * CTA per 128 query rows walks the key rows up to its diagonal.  Inputs as
+ * for lh_attn_bwd_dkdv; dqg out bf16 [B, H, S, d]. */
 lh_status lh_attn_bwd_dq(const lh_config* cfg, const lh_bf16* qg, const lh_bf16* kg,
                          const lh_bf16* vg, const lh_bf16* dog, const float* lse,
                          const float* delta, lh_bf16* dqg, void* stream);
@@ -218,7 +238,9 @@ lh_status lh_attn_bwd_dq(const lh_config* cfg, const lh_bf16* qg, const lh_bf16*
 lh_status lh_scatter(const lh_config* cfg, const lh_bf16* og, const int32_t* slot_map,
                      lh_bf16* o, void* ws, size_t ws_bytes, void* stream);
 
-/* Adjoint of lh_scatter: dog[m] = sum of dO[t] over the shifted range of
+/* Adjoint of lh_scatter (Sec. 3.6 scatter, differentiated as Sec. 3.2
+ * prescribes: the gradient reaches the gathered outputs through stage (iv)):
+ * dog[m] = sum of dO[t] over the shifted range of
  * slot m (clipped to t < N), rounded once to bf16, and delta[m] =
  * rowsum(dog[m] * (og[m] + og_lo[m])) (the D of the attention backward;
  * og_lo may be NULL), both per (b, h).
@@ -228,7 +250,9 @@ lh_status lh_scatter_bwd(const lh_config* cfg, const lh_bf16* dout, const lh_bf1
                          const lh_bf16* og_lo, const int32_t* sel_idx, lh_bf16* dog,
                          float* delta, void* stream);
 
-/* Adjoint of the gather and the mean pooling: dq[t] = sum over levels l of
+/* Adjoint of the gather and the mean pooling (Sec. 3.3 pyramid and Sec. 3.5
+ * gather, differentiated as Sec. 3.2 prescribes: gradients reach Q, K, V
+ * through the gather; the selection carries none): dq[t] = sum over levels l of
  * p^-l dqg[slot(l, floor(t/p^l))] for selected entries (unshifted window),
  * likewise dk and dv.
  *  dq, dk, dv out bf16 [B, N, H, d]                                        */
@@ -236,14 +260,15 @@ lh_status lh_gather_bwd(const lh_config* cfg, const lh_bf16* dqg, const lh_bf16*
                         const lh_bf16* dvg, const int32_t* slot_map, lh_bf16* dq,
                         lh_bf16* dk, lh_bf16* dv, void* stream);
 
-/* Whole layer forward: lh_pyramid, lh_score_topk, lh_gather, lh_attn_fwd,
- * lh_scatter.  o out bf16 [B, N, H, d].  `saved` (>= saved bytes) receives
+/* Whole layer forward, the four stages of Sec. 3.2 in order (Sec. 3.3-3.6):
+ * lh_pyramid, lh_score_topk, lh_gather, lh_attn_fwd, lh_scatter.  o out bf16 [B, N, H, d].  `saved` (>= saved bytes) receives
  * what lh_backward needs; `ws` (>= fwd_ws bytes) is scratch.               */
 lh_status lh_forward(const lh_config* cfg, const lh_bf16* q, const lh_bf16* k,
                      const lh_bf16* v, lh_bf16* o, void* saved, size_t saved_bytes,
                      void* ws, size_t ws_bytes, void* stream);
 
-/* Whole layer backward from the saved buffer of the matching lh_forward:
+/* Whole layer backward from the saved buffer of the matching lh_forward
+ * (Sec. 3.2: through stages (iv), (iii) and the gather, indices frozen):
  * lh_scatter_bwd (which also gives D), lh_attn_bwd_dkdv, lh_attn_bwd_dq,
  * lh_gather_bwd.  dq, dk, dv out bf16
  * [B, N, H, d]; `ws` (>= bwd_ws bytes) is scratch.                          */

@@ -159,3 +159,26 @@ def test_gemm_binding_checks_operand_shapes(L):
     b = torch.empty(256, 64, dtype=torch.bfloat16)
     with pytest.raises(L.LighthouseError):
         L.lh_gemm(c, [(a, b, 64)])      # host tensors are refused before any call
+
+
+def test_grid_limits_rejected_before_launch(L):
+    """(b, h) pairs (times the L-1 segments of the per-level quota) index the
+    y dimension of the selection grids, which stops at 65535: such configs
+    are refused up front (LH_ERR_UNSUPPORTED), not left to fail at launch."""
+    assert L.lh_config_check(L.make_config(1, 4096, 65535, 64, 3, 4, 64)) == 0
+    assert L.lh_config_check(L.make_config(2, 4096, 40000, 64, 3, 4, 64)) == 2
+    assert L.lh_config_check(L.make_config(1, 4096, 40000, 64, 3, 4, 64, select_mode=1)) == 2
+    assert L.lh_config_check(L.make_config(1, 4096, 30000, 64, 3, 4, 64, select_mode=1)) == 0
+
+
+def test_bwd_ws_offsets_fit_the_scratch(L):
+    cfg = L.make_config(2, 2048, 3, 128, 3, 4, 40)
+    _, bwd, _ = L.lh_workspace_bytes(cfg)
+    offs = L.lh_bwd_ws_offsets(cfg)
+    S, d, BH = L.lh_subseq_len(cfg), 128, 6
+    sizes = [BH * S * 4] + [BH * S * d * 2] * 4
+    assert all(o % 256 == 0 for o in offs)
+    spans = sorted(zip(offs, sizes))
+    for (a, n), (b, _) in zip(spans, spans[1:]):
+        assert a + n <= b
+    assert spans[-1][0] + spans[-1][1] <= bwd

@@ -15,8 +15,13 @@ from hierarchical_selection_attention_b200.inputs import make_qkv
 
 pytestmark = pytest.mark.gpu
 
-# B, N, H, d, L, p, k, seed
-SHAPES = [(1, 4096, 2, 64, 3, 4, 64, 0), (2, 2048, 3, 128, 3, 4, 40, 1), (1, 4096, 2, 64, 3, 4, 64, 0)]
+# B, N, H, d, L, p, k, seed, select_mode, select_chunk: every selection mode,
+# with a shape change between calls so no call can lean on the last one's
+# leftovers
+SHAPES = [(1, 4096, 2, 64, 3, 4, 64, 0, 0, 0), (2, 2048, 3, 128, 3, 4, 40, 1, 0, 0),
+          (1, 4096, 2, 64, 3, 4, 64, 0, 1, 0), (1, 8192, 2, 64, 4, 4, 32, 2, 1, 0),
+          (1, 4096, 2, 64, 3, 4, 64, 0, 2, 32), (2, 2048, 3, 128, 3, 4, 40, 1, 2, 20),
+          (1, 4096, 2, 64, 3, 4, 64, 0, 0, 0)]
 
 
 def _scores(L, cfg, q, k, v):
@@ -35,9 +40,9 @@ def test_noalloc_topk_matches_workspace_entry_point():
     from hierarchical_selection_attention_b200 import lighthouse as L
 
     assert L.lh_score_topk_noalloc_max_bytes() == 8 << 20
-    for B, N, H, d, Lv, p, k, seed in SHAPES:
+    for B, N, H, d, Lv, p, k, seed, mode, chunk in SHAPES:
         q, kk, v = (t.cuda() for t in make_qkv(B, N, H, d, seed))
-        cfg = L.make_config(B, N, H, d, Lv, p, k)
+        cfg = L.make_config(B, N, H, d, Lv, p, k, select_mode=mode, select_chunk=chunk)
         S, P = L.lh_subseq_len(cfg), L.lh_total_entries(cfg)
         qk, kq = _scores(L, cfg, q, kk, v)
         fws, _, _ = L.lh_workspace_bytes(cfg)
@@ -60,9 +65,12 @@ def test_noalloc_topk_rejects_shapes_beyond_its_array():
         pytest.skip("needs a CUDA device")
     from hierarchical_selection_attention_b200 import lighthouse as L
 
-    cfg = L.make_config(64, 1 << 20, 8, 128, 3, 4, 1024)   # B*H = 512 heads: ~27 MB of scratch
     x = torch.empty(16, dtype=torch.float32, device="cuda")
     i = torch.empty(16, dtype=torch.int32, device="cuda")
-    with pytest.raises(L.LighthouseError) as e:
-        L.lh_score_topk_noalloc(cfg, x, x, i, i)
-    assert e.value.code == 3  # LH_ERR_WORKSPACE, raised before any launch
+    # B*H = 512 heads: ~27 MB of scratch; and the per-level quota at B*H = 128,
+    # L = 3, N = 2^20, whose two segments per head need ~13 MB
+    for cfg in (L.make_config(64, 1 << 20, 8, 128, 3, 4, 1024),
+                L.make_config(16, 1 << 20, 8, 128, 3, 4, 1024, select_mode=1)):
+        with pytest.raises(L.LighthouseError) as e:
+            L.lh_score_topk_noalloc(cfg, x, x, i, i)
+        assert e.value.code == 3  # LH_ERR_WORKSPACE, raised before any launch
