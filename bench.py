@@ -72,7 +72,7 @@ def algorithmic(w):
         "gather": ("hbm", 6 * gat + B * H * S * 4),
         "attn_fwd": ("tensor", 2 * tri),
         "scatter": ("hbm", gat + tok + B * H * P * 4),
-        "scatter_bwd": ("hbm", tok + 3 * gat + B * H * S * 4),
+        "scatter_bwd": ("hbm", tok + 2 * gat + B * H * S * 4),   # dO, og in; dog, D out
         "attn_bwd_dkdv": ("tensor", 4 * tri),
         "attn_bwd_dq": ("tensor", 1 * tri),    # dS K; S and dP are recomputed (2 more GEMMs)
         "gather_bwd": ("hbm", 3 * gat + 3 * tok + B * H * P * 4),
@@ -168,6 +168,18 @@ def barrier(ws):
 
 
 # ---------------------------------------------------------------- our arm --
+
+def bench_config(args, w, ws):
+    """The workload description both arms print (the driver compares them)."""
+    B, N, H, d, Lv, p, k, S, P, R, C = sizes(w)
+    tok_gib = 3 * B * N * H * d * 2 / 2**30
+    return {"workload": f"{w['name']}: B={B} N={N} H={H} d={d} L={Lv} p={p} k={k} S={S}",
+            "step": "lh_forward + lh_backward stages (fwd+bwd)",
+            "l2": f"inputs larger than L2 ({tok_gib:.2f} GiB of Q,K,V per step); no flush",
+            "parallelism": f"replicas x{ws} (independent layers, no collective)",
+            "selection": SELECT_NAMES[args.select_mode] +
+            (f", {args.select_chunk} per chunk" if args.select_mode == 2 else "")}
+
 
 def run_ours(args, w, ws, rank, local):
     from hierarchical_selection_attention_b200 import lighthouse as L
@@ -342,12 +354,7 @@ def run_ours(args, w, ws, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded: N(0,1) x per-token lognormal(0,0.5), 64 heavy tokens x4)",
-        "config": {"workload": f"{w['name']}: B={B} N={N} H={H} d={d} L={Lv} p={p} k={k} S={S}",
-                   "step": "lh_forward + lh_backward stages (fwd+bwd)",
-                   "l2": "inputs larger than L2 (3 GiB of Q,K,V per step); no flush",
-                   "parallelism": f"replicas x{ws} (independent layers, no collective)",
-                   "selection": SELECT_NAMES[args.select_mode] +
-                   (f", {args.select_chunk} per chunk" if args.select_mode == 2 else "")},
+        "config": bench_config(args, w, ws),
         "fwd_tokens_per_s": ws * B * N / (fwd_ms / 1e3), "fwd_ms": fwd_ms,
         "stages": per_stage, "roofline": roof, "e2e": e2e, "gpu_launches": launches,
         "clocks": clocks,
@@ -420,22 +427,66 @@ def blas_threads() -> int:
     return os.cpu_count() or 1
 
 
+def host_cores() -> dict:
+    """Cores the oracle ran on: its matrix products use the BLAS threads; its
+    element-wise passes, sorts and scans run on one thread."""
+    try:
+        aff = len(os.sched_getaffinity(0))
+    except AttributeError:
+        aff = os.cpu_count() or 1
+    cpu = ""
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                cpu = ln.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return {"blas_threads": blas_threads(), "affinity_cores": aff, "cpu_model": cpu}
+
+
+def oracle_whole_head(wi: int = 1):
+    """One (b, h) head of a workload through the whole oracle, forward and
+    backward over every token and all S gathered rows, timed whole (no
+    sampling, no extrapolation).  Returns (seconds, description)."""
+    from oracle import lighthouse_oracle as lo
+    w = WORKLOADS[wi]
+    B, N, H, d, Lv, p, k, S, P, R, C = sizes(w)
+    q, kk, v = make_qkv(1, N, 1, d, seed=wi)
+    dout = make_dout(1, N, 1, d, seed=wi)
+    qh, kh, vh, doh = (x[0, :, 0, :].double().numpy() for x in (q, kk, v, dout))
+    t0 = time.perf_counter()
+    st = lo.forward_head(qh, kh, vh, Lv, p, k, parity=True)
+    lo.backward_head(st, doh)
+    sec = time.perf_counter() - t0
+    return sec, (f"one (b,h) head of {w['name']} (S={S}) forward+backward through the whole "
+                 f"oracle, timed whole: {sec:.1f} s, i.e. {N / sec:.0f} head-tokens/s")
+
+
 def run_reference(args, w):
-    vals = []
+    """The reference arm: the CPU oracle as it stands.  Each of the warm-up
+    and timed steps is one bounded sample of the workload (oracle_sample);
+    ms_per_step is the measured time of one such sample, and value the
+    whole-workload throughput the sample's work fraction gives."""
+    vals, secs = [], []
     desc = ""
     for i in range(args.warmup + args.steps):
-        tok_s, _, desc = oracle_sample(w, rows_per_head=args.ref_rows, seed=args.workload)
+        tok_s, sec, desc = oracle_sample(w, rows_per_head=args.oracle_rows, seed=args.workload)
         if i >= args.warmup:
             vals.append(tok_s)
+            secs.append(sec)
     v = statistics.median(vals)
-    cores = blas_threads()
+    cores = host_cores()
     return {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": 1e3 * sizes(w)[0] * sizes(w)[1] / v,
+            "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(secs),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded, same recipe)", "impl": "reference",
-            "config": {"workload": w["name"], "arm": "CPU fp64 oracle (numpy), host cores"},
-            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": desc},
+            "config": bench_config(args, w, 1),
+            "arm": "CPU fp64 oracle (numpy) on the host cores; each step is one bounded sample "
+                   "of the workload (cpu_baseline.sample); ms_per_step is the sample's measured "
+                   "time, value the whole-workload tokens/s it extrapolates to",
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores["blas_threads"],
+                             "kind": "oracle", "sample": desc, **cores},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
@@ -566,8 +617,8 @@ def main():
     ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ref-rows", type=int, default=32)
-    ap.add_argument("--cpu-rows", type=int, default=96)
+    ap.add_argument("--oracle-rows", type=int, default=64,
+                    help="query rows per head of the oracle's attention sample (both CPU legs)")
     ap.add_argument("--sweep", action="store_true",
                     help="latency over N = 8K..512K (one JSON line per N) instead of the bench line")
     ap.add_argument("--no-sdpa", action="store_true", help="--sweep without the dense SDPA context")
@@ -590,8 +641,6 @@ def main():
         rank = int(os.environ.get("RANK", "0"))
         if rank != 0:
             return
-        args.steps = min(args.steps, 5)
-        args.warmup = min(args.warmup, 1)
         print(json.dumps(run_reference(args, w)), flush=True)
         return
 
@@ -600,9 +649,14 @@ def main():
         line = run_ours(args, w, ws, rank, local)
         if rank == 0:
             if not args.no_cpu_baseline and ws == 1:
-                tok_s, _, desc = oracle_sample(w, rows_per_head=args.cpu_rows, seed=args.workload)
-                line["cpu_baseline"] = {"value": tok_s, "unit": UNIT, "cores": blas_threads(),
-                                        "kind": "oracle", "sample": desc}
+                tok_s, _, desc = oracle_sample(w, rows_per_head=args.oracle_rows, seed=args.workload)
+                cores = host_cores()
+                line["cpu_baseline"] = {"value": tok_s, "unit": UNIT,
+                                        "cores": cores["blas_threads"], "kind": "oracle",
+                                        "sample": desc, **cores}
+                sec, wdesc = oracle_whole_head(1)
+                line["cpu_baseline"]["whole_head"] = {"seconds": sec, "workload": WORKLOADS[1]["name"],
+                                                      "description": wdesc}
             print(json.dumps(line), flush=True)
     finally:
         if ws > 1:
