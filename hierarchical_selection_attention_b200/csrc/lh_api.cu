@@ -341,6 +341,80 @@ lh_status lh_attn_bwd_dq(const lh_config* cfg, const lh_bf16* qg, const lh_bf16*
                                nullptr, nullptr, D.status, (cudaStream_t)stream, 2));
 }
 
+// ---- ring steps (context parallelism) --------------------------------------
+
+namespace {
+// Mode and flags of one ring step; the accumulators a step reads or keeps
+// must be given, the outputs a closing step writes must be given.
+lh_status ring_args(int32_t mode, int32_t first, int32_t last) {
+  if (mode != LH_BLOCK_DIAG && mode != LH_BLOCK_FULL) return LH_ERR_INVALID_ARGUMENT;
+  if ((first != 0 && first != 1) || (last != 0 && last != 1)) return LH_ERR_INVALID_ARGUMENT;
+  return LH_OK;
+}
+inline bool acc_ok(int32_t first, int32_t last, const void* a) {
+  return (first && last) || (a != nullptr && aligned(a));
+}
+inline bool out_ok(int32_t last, const void* o) { return !last || (o != nullptr && aligned(o)); }
+}  // namespace
+
+lh_status lh_attn_fwd_block(const lh_config* cfg, int32_t mode, int32_t first, int32_t last,
+                            const lh_bf16* qg, const lh_bf16* kg, const lh_bf16* vg,
+                            float* o_acc, float* lse2_acc, lh_bf16* og, lh_bf16* og_lo,
+                            float* lse, void* stream) {
+  LH_TRY(check(cfg));
+  LH_TRY(ring_args(mode, first, last));
+  if (!all_aligned(qg, kg, vg)) return LH_ERR_INVALID_ARGUMENT;
+  if (!acc_ok(first, last, o_acc) || !acc_ok(first, last, lse2_acc)) return LH_ERR_INVALID_ARGUMENT;
+  if (!out_ok(last, og) || !out_ok(last, lse) || (og_lo && !aligned(og_lo)))
+    return LH_ERR_INVALID_ARGUMENT;
+  const LhDims D = launch_dims(cfg);
+  if (!D.status) return LH_ERR_CUDA;
+  return cu(lh_launch_attn_fwd(D.B * D.H, D.S, D.d, D.scale, qg, kg, vg, og, last ? og_lo : nullptr,
+                               lse, D.status, (cudaStream_t)stream, mode == LH_BLOCK_FULL, first,
+                               last, o_acc, lse2_acc));
+}
+
+lh_status lh_attn_bwd_dkdv_block(const lh_config* cfg, int32_t mode, int32_t first,
+                                 int32_t last, const lh_bf16* qg, const lh_bf16* kg,
+                                 const lh_bf16* vg, const lh_bf16* dog, const float* lse,
+                                 const float* delta, float* dk_acc, float* dv_acc, lh_bf16* dkg,
+                                 lh_bf16* dvg, void* stream) {
+  LH_TRY(check(cfg));
+  LH_TRY(ring_args(mode, first, last));
+  if (!all_aligned(qg, kg, vg, dog, lse, delta)) return LH_ERR_INVALID_ARGUMENT;
+  if (!acc_ok(first, last, dk_acc) || !acc_ok(first, last, dv_acc)) return LH_ERR_INVALID_ARGUMENT;
+  if (!out_ok(last, dkg) || !out_ok(last, dvg)) return LH_ERR_INVALID_ARGUMENT;
+  const LhDims D = launch_dims(cfg);
+  if (!D.status) return LH_ERR_CUDA;
+  LhRingStep rs;
+  rs.full = mode == LH_BLOCK_FULL;
+  rs.kv_first = first;
+  rs.kv_last = last;
+  rs.dk_acc = dk_acc;
+  rs.dv_acc = dv_acc;
+  return cu(lh_launch_attn_bwd(D.B * D.H, D.S, D.d, D.scale, qg, kg, vg, dog, lse, delta, nullptr,
+                               dkg, dvg, D.status, (cudaStream_t)stream, 1, &rs));
+}
+
+lh_status lh_attn_bwd_dq_block(const lh_config* cfg, int32_t mode, int32_t first, int32_t last,
+                               const lh_bf16* qg, const lh_bf16* kg, const lh_bf16* vg,
+                               const lh_bf16* dog, const float* lse, const float* delta,
+                               float* dq_acc, lh_bf16* dqg, void* stream) {
+  LH_TRY(check(cfg));
+  LH_TRY(ring_args(mode, first, last));
+  if (!all_aligned(qg, kg, vg, dog, lse, delta)) return LH_ERR_INVALID_ARGUMENT;
+  if (!acc_ok(first, last, dq_acc) || !out_ok(last, dqg)) return LH_ERR_INVALID_ARGUMENT;
+  const LhDims D = launch_dims(cfg);
+  if (!D.status) return LH_ERR_CUDA;
+  LhRingStep rs;
+  rs.full = mode == LH_BLOCK_FULL;
+  rs.q_first = first;
+  rs.q_last = last;
+  rs.dq_acc = dq_acc;
+  return cu(lh_launch_attn_bwd(D.B * D.H, D.S, D.d, D.scale, qg, kg, vg, dog, lse, delta, dqg,
+                               nullptr, nullptr, D.status, (cudaStream_t)stream, 2, &rs));
+}
+
 lh_status lh_scatter(const lh_config* cfg, const lh_bf16* og, const int32_t* slot_map,
                      lh_bf16* o, void* ws, size_t ws_bytes, void* stream) {
   LH_TRY(check(cfg));
@@ -408,6 +482,79 @@ lh_status lh_forward(const lh_config* cfg, const lh_bf16* q, const lh_bf16* k,
   if (cfg->scatter_mode == 1)
     return cu(lh_launch_scatter_atomic(D, og, slot_map, o, at<void>(ws, w.atomic), st, nullptr));
   return cu(lh_launch_scatter(D, og, slot_map, o, st));
+}
+
+// ---- the layer in halves around its attention ------------------------------
+
+lh_status lh_forward_gather(const lh_config* cfg, const lh_bf16* q, const lh_bf16* k,
+                            const lh_bf16* v, void* saved, size_t saved_bytes, void* ws,
+                            size_t ws_bytes, void* stream) {
+  LH_TRY(check(cfg));
+  if (!all_aligned(q, k, v, saved, ws)) return LH_ERR_INVALID_ARGUMENT;
+  const LhDims D = launch_dims(cfg);
+  if (!D.status) return LH_ERR_CUDA;
+  const FwdWs w = fwd_layout(D, cfg->scatter_mode);
+  const Saved s = saved_layout(D);
+  if (ws_bytes < w.total || saved_bytes < s.total) return LH_ERR_WORKSPACE;
+  const cudaStream_t st = (cudaStream_t)stream;
+  int32_t* sel_idx = at<int32_t>(saved, s.off[0]);
+  int32_t* slot_map = at<int32_t>(saved, s.off[1]);
+  lh_bf16* q_lv = at<lh_bf16>(ws, w.q_lv);
+  lh_bf16* k_lv = at<lh_bf16>(ws, w.k_lv);
+  lh_bf16* v_lv = at<lh_bf16>(ws, w.v_lv);
+  float* qk = at<float>(ws, w.qk);
+  float* kq = at<float>(ws, w.kq);
+  LH_TRY(cu(lh_launch_pyramid(D, q, k, v, q_lv, k_lv, v_lv, qk, kq, st)));
+  LH_TRY(cu(lh_launch_select(D, qk, kq, sel_idx, slot_map, at<void>(ws, w.select), st, nullptr)));
+  return cu(lh_launch_gather(D, q, k, v, q_lv, k_lv, v_lv, sel_idx, at<lh_bf16>(saved, s.off[2]),
+                             at<lh_bf16>(saved, s.off[3]), at<lh_bf16>(saved, s.off[4]), st));
+}
+
+lh_status lh_forward_scatter(const lh_config* cfg, const void* saved, size_t saved_bytes,
+                             lh_bf16* o, void* ws, size_t ws_bytes, void* stream) {
+  LH_TRY(check(cfg));
+  if (!all_aligned(saved, o, ws)) return LH_ERR_INVALID_ARGUMENT;
+  const LhDims D = launch_dims(cfg);
+  if (!D.status) return LH_ERR_CUDA;
+  const FwdWs w = fwd_layout(D, cfg->scatter_mode);
+  const Saved s = saved_layout(D);
+  if (ws_bytes < w.total || saved_bytes < s.total) return LH_ERR_WORKSPACE;
+  const cudaStream_t st = (cudaStream_t)stream;
+  const lh_bf16* og = at<lh_bf16>(saved, s.off[5]);
+  const int32_t* slot_map = at<int32_t>(saved, s.off[1]);
+  if (cfg->scatter_mode == 1)
+    return cu(lh_launch_scatter_atomic(D, og, slot_map, o, at<void>(ws, w.atomic), st, nullptr));
+  return cu(lh_launch_scatter(D, og, slot_map, o, st));
+}
+
+lh_status lh_backward_scatter(const lh_config* cfg, const void* saved, size_t saved_bytes,
+                              const lh_bf16* dout, void* ws, size_t ws_bytes, void* stream) {
+  LH_TRY(check(cfg));
+  if (!all_aligned(saved, dout, ws)) return LH_ERR_INVALID_ARGUMENT;
+  const LhDims D = launch_dims(cfg);
+  if (!D.status) return LH_ERR_CUDA;
+  const Saved s = saved_layout(D);
+  const BwdWs b = bwd_layout(D);
+  if (saved_bytes < s.total || ws_bytes < b.total) return LH_ERR_WORKSPACE;
+  return cu(lh_launch_scatter_bwd(D, dout, at<lh_bf16>(saved, s.off[5]),
+                                  at<lh_bf16>(saved, s.off[6]), at<int32_t>(saved, s.off[0]),
+                                  at<lh_bf16>(ws, b.dog), at<float>(ws, b.delta),
+                                  (cudaStream_t)stream));
+}
+
+lh_status lh_backward_gather(const lh_config* cfg, const void* saved, size_t saved_bytes,
+                             const void* ws, size_t ws_bytes, lh_bf16* dq, lh_bf16* dk,
+                             lh_bf16* dv, void* stream) {
+  LH_TRY(check(cfg));
+  if (!all_aligned(saved, ws, dq, dk, dv)) return LH_ERR_INVALID_ARGUMENT;
+  const LhDims D = launch_dims(cfg);
+  if (!D.status) return LH_ERR_CUDA;
+  const Saved s = saved_layout(D);
+  const BwdWs b = bwd_layout(D);
+  if (saved_bytes < s.total || ws_bytes < b.total) return LH_ERR_WORKSPACE;
+  return cu(lh_launch_gather_bwd(D, at<lh_bf16>(ws, b.dqg), at<lh_bf16>(ws, b.dkg),
+                                 at<lh_bf16>(ws, b.dvg), at<int32_t>(saved, s.off[1]), dq, dk, dv,
+                                 (cudaStream_t)stream));
 }
 
 lh_status lh_backward(const lh_config* cfg, const void* saved, size_t saved_bytes,

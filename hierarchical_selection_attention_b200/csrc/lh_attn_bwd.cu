@@ -25,6 +25,14 @@
 // exchange; two warps per SM sub-partition hide each other's latency.)
 // The same shared-memory tile of Q, dO or K serves as a K-major operand in
 // one MMA and as an MN-major operand in another.
+//
+// Ring steps (context parallelism: one shard's query rows against one K/V
+// block of the same length S, see the forward kernel): `full` walks every
+// tile of an earlier shard's block with no mask (rows and keys past S are
+// zero-filled by TMA, so they add nothing); the gradients of a block that
+// several steps reach are summed in fp32 accumulators (`first` writes them
+// without reading, `last` writes the bf16 result instead), in step order,
+// so the sums stay bitwise reproducible.
 #include "lh_sm100.cuh"
 
 namespace {
@@ -37,6 +45,31 @@ using namespace sm100;
 constexpr int kSoftmax = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
+
+// One thread's 32 gradient columns x * mul of a ring step: summed with the
+// fp32 accumulator (unless first), then kept there (unless last) or written
+// as bf16 (last).  acc: 8 float4, out: 4 uint4.
+__device__ __forceinline__ void lh_chain_store(const uint32_t (&o)[32], float mul, float4* acc,
+                                               uint4* out, int first, int last) {
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    float x[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(o[v * 8 + e]) * mul;
+    if (!first) {
+      const float4 a = acc[2 * v], b = acc[2 * v + 1];
+      x[0] += a.x; x[1] += a.y; x[2] += a.z; x[3] += a.w;
+      x[4] += b.x; x[5] += b.y; x[6] += b.z; x[7] += b.w;
+    }
+    if (last) {
+      out[v] = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
+                          pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
+    } else {
+      acc[2 * v] = make_float4(x[0], x[1], x[2], x[3]);
+      acc[2 * v + 1] = make_float4(x[4], x[5], x[6], x[7]);
+    }
+  }
+}
 
 // ------------------------------------------------------------------ dK/dV --
 
@@ -98,7 +131,8 @@ __global__ void __launch_bounds__(kThreadsDkdv, 1)
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                     const float* __restrict__ lse, const float* __restrict__ delta,
                     uint4* __restrict__ dkg, uint4* __restrict__ dvg, int S, int BH, float scale,
-                    int* status) {
+                    int* status, int full, int first, int last, float* __restrict__ dk_acc,
+                    float* __restrict__ dv_acc) {
   using Lay = DkdvLayout<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -108,7 +142,7 @@ __global__ void __launch_bounds__(kThreadsDkdv, 1)
   const int kt = (int)(blockIdx.x / BH);  // key tile 0 walks the most query tiles: first
   const int bh = (int)(blockIdx.x % BH);
   const int n_q = (S + Q_N - 1) / Q_N;
-  const int i0 = kt;                       // the diagonal query tile (Q_N == KV_M)
+  const int i0 = full ? 0 : kt;            // the diagonal query tile (Q_N == KV_M)
   const int n_it = n_q - i0;
 
   if (threadIdx.x == 0) {
@@ -264,7 +298,7 @@ __global__ void __launch_bounds__(kThreadsDkdv, 1)
     bool ok = true;
     for (int it = 0; ok && it < n_it; ++it) {
       const int qc0 = (i0 + it) * Q_N + h * 64;      // first query column of this thread
-      const bool diag = it == 0;
+      const bool diag = !full && it == 0;
       // ---- P = exp2(c (s - LSE / scale)): fp32 kept in registers, bf16 into TMEM
       uint32_t p[64];                                // scores, then P (fp32 bits)
       const uint64_t c2 = f2_pack(c, c);
@@ -329,12 +363,18 @@ __global__ void __launch_bounds__(kThreadsDkdv, 1)
       const int which = h;                           // warpgroup 0 writes dV, 1 writes dK
       uint4* dst = (which ? dkg : dvg) + ((int64_t)bh * S + kvrow) * (HD / 8);
       const float mul = which ? scale : 1.f;
+      const bool chain = !(first && last);
+      float4* acc = chain ? reinterpret_cast<float4*>(which ? dk_acc : dv_acc) +
+                                ((int64_t)bh * S + kvrow) * (HD / 4)
+                          : nullptr;
 #pragma unroll
       for (int cchunk = 0; cchunk < HD / 32; ++cchunk) {
         uint32_t o[32];
         tmem_ld32(tmem + lane_addr + 256 + which * HD + cchunk * 32, o);
         tmem_ld_wait();
-        if (kvrow < S) {
+        if (kvrow < S && chain) {
+          lh_chain_store(o, mul, acc + cchunk * 8, dst + cchunk * 4, first, last);
+        } else if (kvrow < S) {
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
             uint4 w;
@@ -401,7 +441,8 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
     k_attn_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                   const float* __restrict__ lse, const float* __restrict__ delta,
-                  uint4* __restrict__ dqg, int S, int BH, float scale, int* status) {
+                  uint4* __restrict__ dqg, int S, int BH, float scale, int* status, int full,
+                  int first, int last, float* __restrict__ dq_acc) {
   using Lay = DqLayout<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -411,7 +452,7 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
   const int n_qt = (S + Q_M - 1) / Q_M;
   const int qt = n_qt - 1 - (int)(blockIdx.x / BH);  // longest rows first
   const int bh = (int)(blockIdx.x % BH);
-  const int n_kv = qt + 1;                           // key tiles up to the diagonal (KV_N == Q_M)
+  const int n_kv = full ? n_qt : qt + 1;             // key tiles up to the diagonal (KV_N == Q_M)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->qfull, 1);
@@ -539,7 +580,7 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
     for (int j = 0; ok && j < n_kv; ++j) {
       const int sb = j & 1;
       const int kc0 = j * KV_N + h * 64;               // first key column of this thread
-      const bool diag = j == qt;
+      const bool diag = !full && j == qt;
       // ---- P = exp2(c s - lse), fp32 in registers
       uint32_t p[64];
       if (!mbar_wait(&bars->sfull[sb], (j >> 1) & 1, status, 38)) { ok = false; break; }
@@ -595,13 +636,18 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
     if (ok && mbar_wait(&bars->done, 0, status, 40)) {
       tc_fence_after();
       uint4* dst = dqg + ((int64_t)bh * S + qrow) * (HD / 8);
+      const bool chain = !(first && last);
+      float4* acc = chain ? reinterpret_cast<float4*>(dq_acc) + ((int64_t)bh * S + qrow) * (HD / 4)
+                          : nullptr;
 #pragma unroll
       for (int q = 0; q < HD / 64; ++q) {            // each warpgroup: half of the d columns
         const int cchunk = h * (HD / 64) + q;
         uint32_t o[32];
         tmem_ld32(tmem + lane_addr + 384 + cchunk * 32, o);
         tmem_ld_wait();
-        if (qrow < S) {
+        if (qrow < S && chain) {
+          lh_chain_store(o, scale, acc + cchunk * 8, dst + cchunk * 4, first, last);
+        } else if (qrow < S) {
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
             uint4 w;
@@ -632,21 +678,22 @@ static_assert(kSmemDkdv > 232448 / 2 && kSmemDq > 232448 / 2, "one CTA per SM");
 template <int HD>
 cudaError_t launch_hd(int BH, int S, float scale, const CUtensorMap* maps, const float* lse,
                       const float* delta, lh_bf16* dqg, lh_bf16* dkg, lh_bf16* dvg, int* status,
-                      cudaStream_t st, int which) {
+                      cudaStream_t st, int which, const LhRingStep& rs) {
   // maps: Q, K, V, dO with 128-row boxes (every tile of both kernels)
   if (which & 1) {
     cudaFuncSetAttribute(k_attn_bwd_dkdv<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemDkdv);
     const int n_kt = (S + KV_M - 1) / KV_M;
     k_attn_bwd_dkdv<HD><<<n_kt * BH, kThreadsDkdv, kSmemDkdv, st>>>(
         maps[0], maps[1], maps[2], maps[3], lse, delta, (uint4*)dkg, (uint4*)dvg, S, BH, scale,
-        status);
+        status, rs.full, rs.kv_first, rs.kv_last, rs.dk_acc, rs.dv_acc);
   }
   if (which & 2) {
     cudaFuncSetAttribute(k_attn_bwd_dq<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemDq);
     const int n_qt = (S + Q_M - 1) / Q_M;
     k_attn_bwd_dq<HD><<<n_qt * BH, kThreadsDq, kSmemDq, st>>>(maps[0], maps[1], maps[2], maps[3],
                                                              lse, delta, (uint4*)dqg, S, BH, scale,
-                                                             status);
+                                                             status, rs.full, rs.q_first,
+                                                             rs.q_last, rs.dq_acc);
   }
   return cudaGetLastError();
 }
@@ -660,14 +707,16 @@ cudaError_t lh_launch_attn_bwd(int BH, int64_t S, int d, float scale, const lh_b
                                const lh_bf16* kg, const lh_bf16* vg, const lh_bf16* dog,
                                const float* lse, const float* delta, lh_bf16* dqg,
                                lh_bf16* dkg, lh_bf16* dvg, int* status, cudaStream_t st,
-                               int which) {
+                               int which, const LhRingStep* ring) {
+  const LhRingStep plain{};
+  const LhRingStep& rs = ring ? *ring : plain;
   CUtensorMap maps[4];
   const lh_bf16* src[4] = {qg, kg, vg, dog};
   for (int i = 0; i < 4; ++i)
     if (!lh_make_tmap_3d(&maps[i], src[i], BH, S, d, 128)) return cudaErrorInvalidValue;
   if (d == 128)
-    return launch_hd<128>(BH, (int)S, scale, maps, lse, delta, dqg, dkg, dvg, status, st, which);
+    return launch_hd<128>(BH, (int)S, scale, maps, lse, delta, dqg, dkg, dvg, status, st, which, rs);
   if (d == 64)
-    return launch_hd<64>(BH, (int)S, scale, maps, lse, delta, dqg, dkg, dvg, status, st, which);
+    return launch_hd<64>(BH, (int)S, scale, maps, lse, delta, dqg, dkg, dvg, status, st, which, rs);
   return cudaErrorInvalidValue;
 }

@@ -27,6 +27,19 @@
 // (P_h packed into the first 32 columns of its half), O_0 from 256 and O_1
 // from 256 + d.  Shared memory: Q, KST K stages and VST V stages (128 x d
 // bf16 each), 128-byte swizzled, 1024-byte aligned, and the merge buffer.
+//
+// Blocks of a ring (context parallelism, the pages' multi-GPU training
+// note: the gathered sub-sequences of consecutive shards rotate through
+// ring attention).  The same kernel computes one step of it: the rows of
+// one shard's sub-sequence against one K/V block of the same length S,
+// either the shard's own block (causal, as above) or an earlier shard's
+// block (`full`: every key visible; keys past S masked).  Partial results
+// merge by log-sum-exp into fp32 accumulators, in base 2:
+//   lse2 = log2(2^a + 2^b),  O = O_a 2^(a - lse2) + O_b 2^(b - lse2)
+// with a the accumulated and b this block's lse2 and O_a, O_b normalised.
+// `first` writes the accumulators without reading them; `last` writes the
+// bf16 output and natural-log LSE instead of them.  first && last is the
+// plain single-block attention.
 #include <cudaTypedefs.h>
 
 #include "lh_sm100.cuh"
@@ -72,7 +85,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     k_attn_fwd(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, uint4* __restrict__ og,
                uint4* __restrict__ og_lo, float* __restrict__ lse, int S, int BH,
-               float scale_log2, int* status) {
+               float scale_log2, int* status, int full, int first, int last,
+               float* __restrict__ o_acc, float* __restrict__ lse2_acc) {
   using Lay = FwdLayout<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -83,7 +97,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_qt = (S + BM - 1) / BM;
   const int qt = n_qt - 1 - (int)(blockIdx.x / BH);  // longest rows first
   const int bh = (int)(blockIdx.x % BH);
-  const int n_kv = qt + 1;                           // key tiles up to the diagonal (BN == BM)
+  // key tiles up to the diagonal (BN == BM), or all of them for an earlier block
+  const int n_kv = full ? n_qt : qt + 1;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->qfull, 1);
@@ -199,14 +214,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
       tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
       tmem_ld_wait();
-      const bool diag = (j == qt);
+      // masked tile: the diagonal (keys <= r) or, for an earlier block, the
+      // ragged last tile (keys < S); columns c0 + e < lim are kept
+      const bool diag = !full && (j == qt);
+      const bool msk = diag || (full && (j + 1) * BN > S);
+      const int lim = diag ? r + 1 : S - j * BN;
       float mxv[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) mxv[u] = -INFINITY;
-      if (diag) {
+      if (msk) {
 #pragma unroll
         for (int e = 0; e < 64; ++e)
-          if (c0 + e <= r) mxv[e & 7] = fmaxf(mxv[e & 7], __uint_as_float(s[e]));
+          if (c0 + e < lim) mxv[e & 7] = fmaxf(mxv[e & 7], __uint_as_float(s[e]));
       } else {
 #pragma unroll
         for (int e = 0; e < 64; e += 2)
@@ -237,9 +256,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int i = c * 16 + e;
           const float2 x = f2_unpack(f2_fma(f2_pack(__uint_as_float(s[i]), __uint_as_float(s[i + 1])), sc2, nm2));
           float p0 = ex2(x.x), p1 = ex2(x.y);
-          if (diag) {
-            p0 = (c0 + i <= r) ? p0 : 0.f;
-            p1 = (c0 + i + 1 <= r) ? p1 : 0.f;
+          if (msk) {
+            p0 = (c0 + i < lim) ? p0 : 0.f;
+            p1 = (c0 + i + 1 < lim) ? p1 : 0.f;
           }
           rs2[(i >> 1) & 3] = f2_add(rs2[(i >> 1) & 3], f2_pack(p0, p1));
           pk[e >> 1] = pack_bf16x2(p0, p1);
@@ -274,7 +293,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // HD/2 h .. HD/2 h + HD/2 - 1
     float2* mg = reinterpret_cast<float2*>(smem + Lay::merge);
     mg[h * BM + r] = make_float2(m_used, lsum);
-    named_bar(1, 2 * kHalf);
+    const bool chain = !(first && last);             // a ring step that merges
+    const int64_t row_off = (int64_t)bh * S + qrow;
+    const float lse2_a = (chain && !first && qrow < S) ? lse2_acc[row_off] : -INFINITY;
+    named_bar(1, 2 * kHalf);                         // both halves have read lse2_acc
     const float2 o_ml = mg[(h ^ 1) * BM + r];
     if (ok && mbar_wait_w(&bars->pvdone[(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, status, 10)) {
       tc_fence_after();
@@ -284,7 +306,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float a0 = ex2(m0 - m), a1 = ex2(m1 - m);
       const float l = l0 * a0 + l1 * a1;
       const float inv = 1.f / l;
-      const float w0 = a0 * inv, w1 = a1 * inv;
+      float w0 = a0 * inv, w1 = a1 * inv;
+      // ring step: weights of the accumulated and of this block's output
+      float lse2_out = m + __log2f(l), fa = 0.f;
+      if (chain) {
+        const float b = lse2_out;
+        const float mx = fmaxf(lse2_a, b);
+        const float wa = first ? 0.f : ex2(lse2_a - mx), wb = ex2(b - mx);
+        const float z = wa + wb;
+        lse2_out = mx + __log2f(z);
+        fa = wa / z;
+        w0 *= wb / z;
+        w1 *= wb / z;
+      }
       const uint32_t tO0 = tmem + lane_addr + 256, tO1 = tO0 + HD;
 #pragma unroll
       for (int cc = 0; cc < HD / 64; ++cc) {
@@ -295,12 +329,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait();
         if (qrow < S) {
           const int64_t base = ((int64_t)bh * S + qrow) * (HD / 8) + c * 4;
+          float4* acc = chain ? reinterpret_cast<float4*>(o_acc) + row_off * (HD / 4) + c * 8
+                              : nullptr;
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
             float xv[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e)
               xv[e] = __uint_as_float(o0[v * 8 + e]) * w0 + __uint_as_float(o1[v * 8 + e]) * w1;
+            if (chain && !first) {
+              const float4 a = acc[2 * v], b = acc[2 * v + 1];
+              xv[0] += fa * a.x; xv[1] += fa * a.y; xv[2] += fa * a.z; xv[3] += fa * a.w;
+              xv[4] += fa * b.x; xv[5] += fa * b.y; xv[6] += fa * b.z; xv[7] += fa * b.w;
+            }
+            if (!last) {                             // keep the merged fp32 output
+              acc[2 * v] = make_float4(xv[0], xv[1], xv[2], xv[3]);
+              acc[2 * v + 1] = make_float4(xv[4], xv[5], xv[6], xv[7]);
+              continue;
+            }
             uint4 w;
             w.x = pack_bf16x2(xv[0], xv[1]); w.y = pack_bf16x2(xv[2], xv[3]);
             w.z = pack_bf16x2(xv[4], xv[5]); w.w = pack_bf16x2(xv[6], xv[7]);
@@ -318,7 +364,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (h == 0 && qrow < S) lse[(int64_t)bh * S + qrow] = (m + __log2f(l)) * 0.69314718055994531f;
+      if (h == 0 && qrow < S) {
+        if (last) lse[row_off] = lse2_out * 0.69314718055994531f;
+        else lse2_acc[row_off] = lse2_out;
+      }
     }
     tc_fence_before();
   }
@@ -365,7 +414,8 @@ bool lh_make_tmap_3d(CUtensorMap* m, const void* base, int64_t BH, int64_t rows,
 
 cudaError_t lh_launch_attn_fwd(int BH, int64_t S, int d, float scale, const lh_bf16* qg,
                                const lh_bf16* kg, const lh_bf16* vg, lh_bf16* og,
-                               lh_bf16* og_lo, float* lse, int* status, cudaStream_t st) {
+                               lh_bf16* og_lo, float* lse, int* status, cudaStream_t st,
+                               int full, int first, int last, float* o_acc, float* lse2_acc) {
   CUtensorMap tq, tk, tv;
   if (!lh_make_tmap_3d(&tq, qg, BH, S, d, BM) || !lh_make_tmap_3d(&tk, kg, BH, S, d, BN) ||
       !lh_make_tmap_3d(&tv, vg, BH, S, d, BN))
@@ -376,11 +426,13 @@ cudaError_t lh_launch_attn_fwd(int BH, int64_t S, int d, float scale, const lh_b
   if (d == 128) {
     cudaFuncSetAttribute(k_attn_fwd<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     k_attn_fwd<128><<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, (uint4*)og, (uint4*)og_lo, lse,
-                                                         (int)S, BH, scale_log2, status);
+                                                         (int)S, BH, scale_log2, status, full,
+                                                         first, last, o_acc, lse2_acc);
   } else if (d == 64) {
     cudaFuncSetAttribute(k_attn_fwd<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     k_attn_fwd<64><<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, (uint4*)og, (uint4*)og_lo, lse,
-                                                        (int)S, BH, scale_log2, status);
+                                                        (int)S, BH, scale_log2, status, full,
+                                                        first, last, o_acc, lse2_acc);
   } else {
     return cudaErrorInvalidValue;
   }

@@ -106,9 +106,24 @@ cudaError_t lh_launch_scatter_bwd(const LhDims& D, const lh_bf16* dout, const lh
 cudaError_t lh_launch_gather_bwd(const LhDims& D, const lh_bf16* dqg, const lh_bf16* dkg,
                                  const lh_bf16* dvg, const int32_t* slot_map, lh_bf16* dq,
                                  lh_bf16* dk, lh_bf16* dv, cudaStream_t st);
+// full: the K/V block is an earlier shard's (every key visible); first /
+// last: see the ring-step merge in lh_attn_fwd.cu.  The plain layer passes
+// full = 0, first = last = 1 and no accumulators.
 cudaError_t lh_launch_attn_fwd(int BH, int64_t S, int d, float scale, const lh_bf16* qg,
                                const lh_bf16* kg, const lh_bf16* vg, lh_bf16* og,
-                               lh_bf16* og_lo, float* lse, int* status, cudaStream_t st);
+                               lh_bf16* og_lo, float* lse, int* status, cudaStream_t st,
+                               int full = 0, int first = 1, int last = 1,
+                               float* o_acc = nullptr, float* lse2_acc = nullptr);
+// One ring step of the attention backward: the mode, and for each side (the
+// query rows' dQ; the key block's dK, dV) whether this step opens or closes
+// its fp32 sum.  Zero-initialised it is the plain single-block backward.
+struct LhRingStep {
+  int full = 0;
+  int q_first = 1, q_last = 1, kv_first = 1, kv_last = 1;
+  float* dq_acc = nullptr;
+  float* dk_acc = nullptr;
+  float* dv_acc = nullptr;
+};
 cudaError_t lh_launch_attn_delta(int BH, int64_t S, int d, const lh_bf16* og,
                                  const lh_bf16* og_lo, const lh_bf16* dog, float* delta,
                                  cudaStream_t st);
@@ -117,7 +132,7 @@ cudaError_t lh_launch_attn_bwd(int BH, int64_t S, int d, float scale, const lh_b
                                const lh_bf16* kg, const lh_bf16* vg, const lh_bf16* dog,
                                const float* lse, const float* delta, lh_bf16* dqg,
                                lh_bf16* dkg, lh_bf16* dvg, int* status, cudaStream_t st,
-                               int which);
+                               int which, const LhRingStep* ring = nullptr);
 
 // One warp waiting on an mbarrier nothing completes (lh_selftest.cu).
 cudaError_t lh_launch_wait_timeout_check(int* status, int where, cudaStream_t st);

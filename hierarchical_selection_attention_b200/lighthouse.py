@@ -72,11 +72,18 @@ def _load():
         "lh_attn_bwd": (I32, [C, P, P, P, P, P, P, P, P, P, P, P, SZ, P]),
         "lh_attn_bwd_dkdv": (I32, [C, P, P, P, P, P, P, P, P, P]),
         "lh_attn_bwd_dq": (I32, [C, P, P, P, P, P, P, P, P]),
+        "lh_attn_fwd_block": (I32, [C, I32, I32, I32, P, P, P, P, P, P, P, P, P]),
+        "lh_attn_bwd_dkdv_block": (I32, [C, I32, I32, I32, P, P, P, P, P, P, P, P, P, P, P]),
+        "lh_attn_bwd_dq_block": (I32, [C, I32, I32, I32, P, P, P, P, P, P, P, P, P]),
         "lh_scatter": (I32, [C, P, P, P, P, SZ, P]),
         "lh_scatter_bwd": (I32, [C, P, P, P, P, P, P, P]),
         "lh_gather_bwd": (I32, [C, P, P, P, P, P, P, P, P]),
         "lh_forward": (I32, [C, P, P, P, P, P, SZ, P, SZ, P]),
         "lh_backward": (I32, [C, P, SZ, P, P, P, P, P, SZ, P]),
+        "lh_forward_gather": (I32, [C, P, P, P, P, SZ, P, SZ, P]),
+        "lh_forward_scatter": (I32, [C, P, SZ, P, P, SZ, P]),
+        "lh_backward_scatter": (I32, [C, P, SZ, P, P, SZ, P]),
+        "lh_backward_gather": (I32, [C, P, SZ, P, SZ, P, P, P, P]),
         "lh_check_wait_timeout": (I32, [P]),
         "lh_get_device_status": (I32, [P, ctypes.POINTER(I32)]),
         "lh_status_string": (ctypes.c_char_p, [I32]),
@@ -96,8 +103,12 @@ _lib = _load()
 EXPORTED = ("lh_config_check", "lh_subseq_len", "lh_total_entries", "lh_pooled_rows",
             "lh_workspace_bytes", "lh_saved_offsets", "lh_bwd_ws_offsets", "lh_pyramid", "lh_score_topk",
             "lh_score_topk_noalloc", "lh_score_topk_noalloc_max_bytes", "lh_gather",
-            "lh_attn_fwd", "lh_attn_bwd", "lh_attn_bwd_dkdv", "lh_attn_bwd_dq", "lh_scatter", "lh_scatter_bwd", "lh_gather_bwd",
-            "lh_forward", "lh_backward", "lh_check_wait_timeout", "lh_get_device_status",
+            "lh_attn_fwd", "lh_attn_bwd", "lh_attn_bwd_dkdv", "lh_attn_bwd_dq",
+            "lh_attn_fwd_block", "lh_attn_bwd_dkdv_block", "lh_attn_bwd_dq_block",
+            "lh_scatter", "lh_scatter_bwd", "lh_gather_bwd",
+            "lh_forward", "lh_backward", "lh_forward_gather", "lh_forward_scatter",
+            "lh_backward_scatter", "lh_backward_gather", "lh_check_wait_timeout",
+            "lh_get_device_status",
             "lh_status_string",
             "lh_forward_launches", "lh_backward_launches", "lh_gemm_ws_bytes", "lh_gemm")
 
@@ -238,6 +249,34 @@ def lh_attn_bwd_dq(cfg, qg, kg, vg, dog, lse, delta, dqg, stream=None):
                             _stream(stream)), "lh_attn_bwd_dq")
 
 
+LH_BLOCK_DIAG, LH_BLOCK_FULL = 0, 1
+
+
+def lh_attn_fwd_block(cfg, mode, first, last, qg, kg, vg, o_acc, lse2_acc, og, lse, og_lo=None,
+                      stream=None):
+    _ck(_lib.lh_attn_fwd_block(ctypes.byref(cfg), mode, int(first), int(last), _p(qg, BF16),
+                               _p(kg, BF16), _p(vg, BF16), _p(o_acc, F32), _p(lse2_acc, F32),
+                               _p(og, BF16), _p(og_lo, BF16), _p(lse, F32), _stream(stream)),
+        "lh_attn_fwd_block")
+
+
+def lh_attn_bwd_dkdv_block(cfg, mode, first, last, qg, kg, vg, dog, lse, delta, dk_acc, dv_acc,
+                           dkg, dvg, stream=None):
+    _ck(_lib.lh_attn_bwd_dkdv_block(ctypes.byref(cfg), mode, int(first), int(last), _p(qg, BF16),
+                                    _p(kg, BF16), _p(vg, BF16), _p(dog, BF16), _p(lse, F32),
+                                    _p(delta, F32), _p(dk_acc, F32), _p(dv_acc, F32),
+                                    _p(dkg, BF16), _p(dvg, BF16), _stream(stream)),
+        "lh_attn_bwd_dkdv_block")
+
+
+def lh_attn_bwd_dq_block(cfg, mode, first, last, qg, kg, vg, dog, lse, delta, dq_acc, dqg,
+                         stream=None):
+    _ck(_lib.lh_attn_bwd_dq_block(ctypes.byref(cfg), mode, int(first), int(last), _p(qg, BF16),
+                                  _p(kg, BF16), _p(vg, BF16), _p(dog, BF16), _p(lse, F32),
+                                  _p(delta, F32), _p(dq_acc, F32), _p(dqg, BF16), _stream(stream)),
+        "lh_attn_bwd_dq_block")
+
+
 def lh_scatter(cfg, og, slot_map, o, ws=None, stream=None):
     nb = 0 if ws is None else ws.numel() * ws.element_size()
     _ck(_lib.lh_scatter(ctypes.byref(cfg), _p(og, BF16), _p(slot_map, I32), _p(o, BF16),
@@ -266,6 +305,32 @@ def lh_backward(cfg, saved, dout, dq, dk, dv, ws, stream=None):
     _ck(_lib.lh_backward(ctypes.byref(cfg), _p(saved), saved.numel() * saved.element_size(),
                          _p(dout, BF16), _p(dq, BF16), _p(dk, BF16), _p(dv, BF16), _p(ws),
                          ws.numel() * ws.element_size(), _stream(stream)), "lh_backward")
+
+
+def _nb(t):
+    return t.numel() * t.element_size()
+
+
+def lh_forward_gather(cfg, q, k, v, saved, ws, stream=None):
+    _ck(_lib.lh_forward_gather(ctypes.byref(cfg), _p(q, BF16), _p(k, BF16), _p(v, BF16),
+                               _p(saved), _nb(saved), _p(ws), _nb(ws), _stream(stream)),
+        "lh_forward_gather")
+
+
+def lh_forward_scatter(cfg, saved, o, ws, stream=None):
+    _ck(_lib.lh_forward_scatter(ctypes.byref(cfg), _p(saved), _nb(saved), _p(o, BF16), _p(ws),
+                                _nb(ws), _stream(stream)), "lh_forward_scatter")
+
+
+def lh_backward_scatter(cfg, saved, dout, ws, stream=None):
+    _ck(_lib.lh_backward_scatter(ctypes.byref(cfg), _p(saved), _nb(saved), _p(dout, BF16),
+                                 _p(ws), _nb(ws), _stream(stream)), "lh_backward_scatter")
+
+
+def lh_backward_gather(cfg, saved, ws, dq, dk, dv, stream=None):
+    _ck(_lib.lh_backward_gather(ctypes.byref(cfg), _p(saved), _nb(saved), _p(ws), _nb(ws),
+                                _p(dq, BF16), _p(dk, BF16), _p(dv, BF16), _stream(stream)),
+        "lh_backward_gather")
 
 
 def lh_get_device_status(stream=None):

@@ -230,6 +230,55 @@ lh_status lh_attn_bwd_dq(const lh_config* cfg, const lh_bf16* qg, const lh_bf16*
                          const lh_bf16* vg, const lh_bf16* dog, const float* lse,
                          const float* delta, lh_bf16* dqg, void* stream);
 
+/* ---- ring attention steps (context parallelism) ----
+ * The pages' multi-GPU training note (single-B200 latency paragraph of the
+ * experiments, with App. D.4 cited): the sequence is cut into contiguous
+ * shards, pyramid pooling, scoring and top-k run shard-locally, and the
+ * gathered sub-sequences go through ring attention.  Every entry of shard
+ * r' < r ends before any entry of shard r, so over the shards'
+ * sub-sequences concatenated in shard order the plain causal mask applies:
+ * shard r's rows see all of every earlier shard's block and their own
+ * block causally.  One step is one (query shard, K/V block) pair; `cfg` is
+ * the config of one shard (N = its tokens), so every block has S rows.
+ *  mode   LH_BLOCK_DIAG: the shard's own block (causal);
+ *         LH_BLOCK_FULL: an earlier shard's block (every key visible).
+ *  first  1: this step opens the sum (accumulators written, not read).
+ *  last   1: this step closes it (the bf16 results are written instead of
+ *         the accumulators).  first = last = 1 is the plain single-block
+ *         call, and then the accumulators may be NULL.
+ * Accumulators are fp32 and owned by the caller; steps that share them must
+ * run in order (e.g. on one stream).  Sums run in step order, so results
+ * are bitwise reproducible.  Invalid mode, flags or a missing pointer:
+ * LH_ERR_INVALID_ARGUMENT before any launch. */
+#define LH_BLOCK_DIAG 0
+#define LH_BLOCK_FULL 1
+
+/* Forward step: the partial softmax attention of qg [B,H,S,d] against the
+ * block kg, vg [B,H,S,d] merges into o_acc (fp32 [B,H,S,d], normalised
+ * output so far) and lse2_acc (fp32 [B,H,S], base-2 log-sum-exp so far) by
+ * log-sum-exp.  On the last step og, og_lo (may be NULL) and lse (natural
+ * log) are written as by lh_attn_fwd. */
+lh_status lh_attn_fwd_block(const lh_config* cfg, int32_t mode, int32_t first, int32_t last,
+                            const lh_bf16* qg, const lh_bf16* kg, const lh_bf16* vg,
+                            float* o_acc, float* lse2_acc, lh_bf16* og, lh_bf16* og_lo,
+                            float* lse, void* stream);
+
+/* Backward step, the block's side: this query shard's share of dK, dV of
+ * the block (the query rows' final lse and delta = D), added to dk_acc,
+ * dv_acc (fp32 [B,H,S,d]); the closing step writes dkg, dvg (bf16). */
+lh_status lh_attn_bwd_dkdv_block(const lh_config* cfg, int32_t mode, int32_t first,
+                                 int32_t last, const lh_bf16* qg, const lh_bf16* kg,
+                                 const lh_bf16* vg, const lh_bf16* dog, const float* lse,
+                                 const float* delta, float* dk_acc, float* dv_acc, lh_bf16* dkg,
+                                 lh_bf16* dvg, void* stream);
+
+/* Backward step, the query side: the block's share of dQ of the query
+ * shard, added to dq_acc (fp32 [B,H,S,d]); the closing step writes dqg. */
+lh_status lh_attn_bwd_dq_block(const lh_config* cfg, int32_t mode, int32_t first, int32_t last,
+                               const lh_bf16* qg, const lh_bf16* kg, const lh_bf16* vg,
+                               const lh_bf16* dog, const float* lse, const float* delta,
+                               float* dq_acc, lh_bf16* dqg, void* stream);
+
 /* (iv) scatter-back, Sec. 3.6: o[t] = sum over levels l of og[slot] for the
  * selected entry (l, i) with (i+1) p^l - 1 <= t <= (i+2) p^l - 2, i.e.
  * i = floor((t+1)/p^l) - 1; levels are summed in ascending order in fp32 and
@@ -275,6 +324,36 @@ lh_status lh_forward(const lh_config* cfg, const lh_bf16* q, const lh_bf16* k,
 lh_status lh_backward(const lh_config* cfg, const void* saved, size_t saved_bytes,
                       const lh_bf16* dout, lh_bf16* dq, lh_bf16* dk, lh_bf16* dv,
                       void* ws, size_t ws_bytes, void* stream);
+
+/* ---- the layer in halves around its attention ----
+ * lh_forward = lh_forward_gather, lh_attn_fwd on the saved qg/kg/vg (into
+ * the saved og/og_lo/lse), lh_forward_scatter; lh_backward =
+ * lh_backward_scatter, the attention backward from the bwd_ws dog/delta
+ * into the bwd_ws dqg/dkg/dvg (lh_bwd_ws_offsets), lh_backward_gather.
+ * Same buffers, sizes and errors as lh_forward / lh_backward.  Splitting the
+ * layer there lets another schedule of the attention run in the middle:
+ * ring attention over the shards of a sequence (lh_attn_*_block). */
+
+/* Stages (i)-(iii) up to the gather (Sec. 3.3-3.5): pyramid, scores,
+ * selection and order, gather into the saved qg, kg, vg; sel_idx and
+ * slot_map into the saved buffer. */
+lh_status lh_forward_gather(const lh_config* cfg, const lh_bf16* q, const lh_bf16* k,
+                            const lh_bf16* v, void* saved, size_t saved_bytes, void* ws,
+                            size_t ws_bytes, void* stream);
+
+/* Stage (iv) (Sec. 3.6): scatter of the saved og into o [B, N, H, d]. */
+lh_status lh_forward_scatter(const lh_config* cfg, const void* saved, size_t saved_bytes,
+                             lh_bf16* o, void* ws, size_t ws_bytes, void* stream);
+
+/* Adjoint of stage (iv) (Sec. 3.2, 3.6): dog and delta = D into bwd_ws. */
+lh_status lh_backward_scatter(const lh_config* cfg, const void* saved, size_t saved_bytes,
+                              const lh_bf16* dout, void* ws, size_t ws_bytes, void* stream);
+
+/* Adjoint of the gather and pooling (Sec. 3.2, 3.3, 3.5): the bwd_ws dqg,
+ * dkg, dvg into dq, dk, dv [B, N, H, d]. */
+lh_status lh_backward_gather(const lh_config* cfg, const void* saved, size_t saved_bytes,
+                             const void* ws, size_t ws_bytes, lh_bf16* dq, lh_bf16* dk,
+                             lh_bf16* dv, void* stream);
 
 /* ---- plain GEMMs for the projections around the layer (Sec. 3.1: per-head
  * Q, K, V come from the layer's own W_Q, W_K, W_V; an output projection

@@ -1,0 +1,127 @@
+"""The context-parallel layer on one GPU (ring.LighthouseRingLayer): R shards
+of the sequence, each running stages (i)-(iii) and (iv) on its own tokens,
+the ring attention over their gathered sub-sequences in the ring's step
+order through the library's ring-step kernels (lh_attn_fwd_block,
+lh_attn_bwd_dq_block, lh_attn_bwd_dkdv_block), compared with the oracle's
+context-parallel layer (cp_forward_head / cp_backward_head: the pages'
+multi-GPU training note, shard-local pyramid, scores and top-k, attention
+over the shards' sub-sequences in shard order).
+
+Selection, order and slot map: bit for bit per shard.  Floats: the stated
+bar (max-abs 2e-2 on the envelope-scaled error, rel-L2 5e-3), recorded."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import lighthouse_oracle as lo
+from tests.parity import assert_close, attn_envelopes_full, head, record
+from hierarchical_selection_attention_b200.inputs import make_dout, make_qkv
+
+pytestmark = pytest.mark.gpu
+
+LSE_ABS = 1e-3
+
+# B, N, H, d, L, p, k, R, seed; S per shard: 256 (two full tiles), 288 and 296
+# (ragged last tiles: the earlier blocks' masked key tail), 9216 (the 64K
+# workload's shape cut in four)
+CASES = [(1, 4096, 2, 64, 3, 4, 16, 2, 0), (1, 6144, 2, 128, 3, 4, 20, 3, 1),
+         (2, 4096, 3, 64, 2, 4, 10, 4, 2), (1, 65536, 8, 128, 3, 4, 1024, 4, 3)]
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from hierarchical_selection_attention_b200 import lighthouse, ring
+    return lighthouse, ring
+
+
+def _run(ring, B, N, H, d, Lv, p, k, R, q, kk, v, dout):
+    layer = ring.LighthouseRingLayer(B, N, H, d, Lv, p, k, R)
+    o = layer.forward(q, kk, v)
+    grads = layer.backward(dout)
+    torch.cuda.synchronize()
+    return layer, o, grads
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_ring_layer_matches_oracle(lib, case):
+    L, ring = lib
+    B, N, H, d, Lv, p, k, R, seed = case
+    qh, kh, vh = make_qkv(B, N, H, d, seed=seed)
+    doh = make_dout(B, N, H, d, seed=seed)
+    q, kk, v, dout = (t.cuda() for t in (qh, kh, vh, doh))
+    layer, o, (dq, dk, dv) = _run(ring, B, N, H, d, Lv, p, k, R, q, kk, v, dout)
+    L.check_device_status()
+    Ns, Sr = N // R, layer.S
+    heads = [(b, h) for b in range(B) for h in range(H)]
+    if N >= 65536:
+        heads = [(0, 5)]                       # one head at the large shape
+    for b, h in heads:
+        tag = f"R={R} N={N} [b={b},h={h}]"
+        qx, kx, vx, dox = (head(x, b, h) for x in (qh, kh, vh, doh))
+        st = lo.cp_forward_head(qx, kx, vx, Lv, p, k, R, parity=True)
+        for r, sh in enumerate(st["shards"]):
+            sv = layer.shards[r].views()
+            np.testing.assert_array_equal(sv["sel_idx"][b, h].cpu().numpy(), sh["sel_idx"])
+            np.testing.assert_array_equal(sv["slot_map"][b, h].cpu().numpy(), sh["slot_map"])
+        scale = st["scale"]
+        dog = np.concatenate([lo.round_bf16(lo.scatter_bwd(dox[r * Ns:(r + 1) * Ns], sh["sel_idx"],
+                                                           Ns, Lv, p))
+                              for r, sh in enumerate(st["shards"])])
+        dqg, dkg, dvg = lo.attention_bwd(st["qg"], st["kg"], st["vg"], dog, scale)
+        eo, eq, ek, ev = attn_envelopes_full(st["qg"], st["kg"], st["vg"], dog, scale)
+        cat = lambda key, views: np.concatenate(
+            [views(r)[key][b, h].double().cpu().numpy() for r in range(R)])
+        fv = lambda r: layer.shards[r].views()
+        bv = lambda r: layer.shards[r].bwd_views()
+        assert_close(cat("og", fv), st["og"], f"ring og {tag}", env=eo)
+        lse = cat("lse", fv)
+        record(lse, st["lse"], f"ring lse {tag}")
+        assert np.max(np.abs(lse - st["lse"])) <= LSE_ABS
+        assert_close(cat("dog", bv), dog, f"ring dog {tag}")
+        assert_close(cat("dqg", bv), dqg, f"ring dqg {tag}", env=eq)
+        assert_close(cat("dkg", bv), dkg, f"ring dkg {tag}", env=ek)
+        assert_close(cat("dvg", bv), dvg, f"ring dvg {tag}", env=ev)
+        # token outputs: each shard's scatter and gather adjoint
+        want = lo.cp_backward_head(st, dox)
+        env_o = np.concatenate([lo.scatter(eo[r * Sr:(r + 1) * Sr], sh["slot_map"], Ns, Lv, p)
+                                for r, sh in enumerate(st["shards"])])
+        assert_close(o[b, :, h, :].double().cpu().numpy(), st["o"], f"ring O {tag}", env=env_o)
+        for name, gpu, w, env in (("dQ", dq, want[0], eq), ("dK", dk, want[1], ek),
+                                  ("dV", dv, want[2], ev)):
+            env_t = np.concatenate([lo.pyramid_bwd(env[r * Sr:(r + 1) * Sr], sh["slot_map"], Ns,
+                                                   Lv, p)
+                                    for r, sh in enumerate(st["shards"])])
+            assert_close(gpu[b, :, h, :].double().cpu().numpy(), w, f"ring {name} {tag}", env=env_t)
+
+
+def test_one_shard_ring_is_the_plain_layer_bit_for_bit(lib):
+    L, ring = lib
+    B, N, H, d, Lv, p, k = 1, 4096, 2, 128, 3, 4, 40
+    qh, kh, vh = make_qkv(B, N, H, d, seed=7)
+    doh = make_dout(B, N, H, d, seed=7)
+    q, kk, v, dout = (t.cuda() for t in (qh, kh, vh, doh))
+    _, o1, g1 = _run(ring, B, N, H, d, Lv, p, k, 1, q, kk, v, dout)
+    plain = L.LighthouseLayer(B, N, H, d, Lv, p, k)
+    o0 = plain.forward(q, kk, v)
+    g0 = plain.backward(dout)
+    torch.cuda.synchronize()
+    L.check_device_status()
+    assert torch.equal(o0, o1)
+    for a, b in zip(g0, g1):
+        assert torch.equal(a, b)
+
+
+def test_ring_layer_is_deterministic(lib):
+    L, ring = lib
+    B, N, H, d, Lv, p, k, R = 1, 6144, 2, 128, 3, 4, 20, 3
+    qh, kh, vh = make_qkv(B, N, H, d, seed=4)
+    doh = make_dout(B, N, H, d, seed=4)
+    q, kk, v, dout = (t.cuda() for t in (qh, kh, vh, doh))
+    _, oa, ga = _run(ring, B, N, H, d, Lv, p, k, R, q, kk, v, dout)
+    _, ob, gb = _run(ring, B, N, H, d, Lv, p, k, R, q, kk, v, dout)
+    L.check_device_status()
+    assert torch.equal(oa, ob)
+    for a, b in zip(ga, gb):
+        assert torch.equal(a, b)
