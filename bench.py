@@ -608,6 +608,52 @@ def run_full_layer(args, w):
             "config": {"workload": w["name"], "d_model": Dm}}
 
 
+def run_ring(args, w):
+    """The context-parallel layer with R shards on one GPU
+    (ring.LighthouseRingLayer): shard-local stages (i)-(iii) and (iv), ring
+    attention over the shards' gathered sub-sequences through the ring-step
+    kernels.  One JSON line: forward and forward+backward tokens/s, and the
+    ring attention's algorithmic TFLOP/s (R causal blocks of S rows and
+    R (R - 1) / 2 full S x S blocks, fwd 2 GEMMs, bwd 5 algorithmic)."""
+    from hierarchical_selection_attention_b200 import lighthouse as L, ring
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    B, N, H, d, Lv, p, k = (w[x] for x in ("B", "N", "H", "d", "L", "p", "k"))
+    R = args.ring
+    q, kk, v = (t.to(dev) for t in make_qkv(B, N, H, d, seed=args.workload))
+    dout = make_dout(B, N, H, d, seed=args.workload).to(dev)
+    layer = ring.LighthouseRingLayer(B, N, H, d, Lv, p, k, R, device=dev)
+    o = torch.empty_like(q)
+    grads = tuple(torch.empty_like(q) for _ in range(3))
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / args.steps
+
+    fwd_ms = timed(lambda: layer.forward(q, kk, v, out=o))
+    ms = timed(lambda: (layer.forward(q, kk, v, out=o), layer.backward(dout, grads=grads)))
+    L.check_device_status()
+    S = layer.S
+    one = 2 * B * H * d                                  # FLOP per (row, key) per GEMM
+    pairs = R * S * (S + 1) / 2 + R * (R - 1) / 2 * S * S
+    return {"metric": f"context-parallel Lighthouse layer, {R} shards on 1 B200, fwd+bwd tokens/s",
+            "value": B * N / (ms / 1e3), "unit": UNIT, "ms_per_step": ms, "fwd_ms": fwd_ms,
+            "fwd_tokens_per_s": B * N / (fwd_ms / 1e3), "steps": args.steps, "warmup": args.warmup,
+            "dtype": "bf16", "ring_attention_flop_fwd": 2 * one * pairs,
+            "ring_attention_flop_bwd": 5 * one * pairs,
+            "config": {"workload": w["name"], "shards": R, "shard_tokens": N // R,
+                       "S_per_shard": S}}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -626,6 +672,8 @@ def main():
                     help="selection: 0 joint top-k (default), 1 per-level quota, 2 stratified")
     ap.add_argument("--select-chunk", type=int, default=0,
                     help="per-chunk quota m of the stratified selection")
+    ap.add_argument("--ring", type=int, default=0,
+                    help="time the context-parallel layer with this many shards on one GPU")
     ap.add_argument("--full-layer", action="store_true",
                     help="time the layer with its Q/K/V/output projections (one JSON line)")
     args = ap.parse_args()
@@ -635,6 +683,9 @@ def main():
         return
     if args.full_layer:
         print(json.dumps(run_full_layer(args, w)), flush=True)
+        return
+    if args.ring:
+        print(json.dumps(run_ring(args, w)), flush=True)
         return
 
     if args.impl == "reference":
