@@ -35,7 +35,6 @@ lh_status check(const lh_config* c) {
     w *= c->p;
   }
   if (c->N % w) return LH_ERR_INVALID_ARGUMENT;  // Sec. 3.3: p^(L-1) | N
-  if (w > 65536) return LH_ERR_UNSUPPORTED;      // coarsest window: one selection-mask window
   int64_t cand = 0, P = 0, span = 1;
   for (int l = 0; l < c->L; ++l) {
     P += c->N / span;
@@ -678,7 +677,8 @@ lh_status lh_score_topk_noalloc(const lh_config* cfg, const float* qk, const flo
   if (lh_select_ws_bytes(D) > kNoAllocScratchBytes) return LH_ERR_WORKSPACE;
   void* scratch = topk_scratch_ptr();
   if (!scratch) return LH_ERR_CUDA;
-  // lh_launch_select writes every per-segment threshold before reading it.
+  // lh_launch_select zeroes the histograms it accumulates into before use;
+  // the state and block counts are written before they are read.
   return cu(lh_launch_select(D, qk, kq, sel_idx, slot_map, scratch, (cudaStream_t)stream,
                              nullptr));
 }
@@ -688,7 +688,9 @@ size_t lh_score_topk_noalloc_max_bytes(void) { return kNoAllocScratchBytes; }
 int32_t lh_forward_launches(const lh_config* cfg) {
   if (check(cfg) != LH_OK) return -1;
   const LhDims D = dims(cfg);
-  const int select = 1;   // selection and order: one cluster kernel (lh_select.cu)
+  // kernels only (the memsets of the scratch are copy-engine work, not counted)
+  // hist/find pairs (one fused chunk kernel when stratified) + order count/scan/emit
+  const int select = D.select_mode == 2 ? 1 + 3 : (D.n_cand > 0 ? 12 + 3 : 1 + 3);
   const int scatter = cfg->scatter_mode == 1 ? 2 : 1;
   return 1 + select + 1 + 1 + scatter;
 }

@@ -30,29 +30,8 @@
 // for each, the levels whose entries end at t ((t+1) mod p^l == 0) in
 // ascending order lists the selected entries in exactly that order, so slots
 // come from a prefix sum over t of the number of selected entries ending at
-// t; the emit pass writes sel_idx (slot -> entry) and slot_map (entry ->
-// slot or -1).
-//
-// One launch does all of it.  Each (b, h) gets one thread-block cluster of
-// kCl CTAs; CTA c owns a contiguous range of base tokens (a multiple of
-// p^(L-1) long) and, at every level, the entries that end inside it.
-//  Selection (modes 0, 1): per radix pass every CTA counts the digits of
-//   its own keys in shared memory; after a cluster barrier the leader CTA
-//   sums the kCl histograms through distributed shared memory, picks the
-//   digit and publishes the new state; after a second barrier every CTA
-//   reads it.  Keys are re-read from global memory each pass (they stay in
-//   L2).  Mode 2: the cluster's CTAs share out the head's chunks, each chunk
-//   selected by one CTA with a shared-memory histogram.
-//  Order: every CTA marks which of its entries are selected in shared-memory
-//   bit masks (level by level, for a window of at most kWin tokens at a
-//   time), counts them, takes its first slot from the counts of the
-//   lower-ranked CTAs (read through distributed shared memory) and emits its
-//   tokens in order from the masks.
-// The cluster barriers are hardware barriers that every thread of every CTA
-// reaches (all control flow around them is uniform across the cluster), so
-// nothing spins on memory.  Integer work only: the result is bit-exact and
-// the same on every run.
-#include <cooperative_groups.h>
+// t: a counting pass per block of tokens, a scan over blocks, and an emit
+// pass that writes sel_idx (slot -> entry) and slot_map (entry -> slot or -1).
 #include <cub/block/block_reduce.cuh>
 #include <cub/block/block_scan.cuh>
 
@@ -72,16 +51,9 @@ struct SelState {
   int pad;
 };
 
-constexpr int kSelThreads = 512;
-constexpr int kWarps = kSelThreads / 32;
-constexpr int kBinsPer = kBins / kSelThreads;         // digits per thread in a find step
-constexpr int kUnroll = 8;                            // keys in flight per thread
-constexpr int kItems = 4;                             // tokens per thread per emit tile
-constexpr int kTile = kSelThreads * kItems;
-constexpr int64_t kWin = 65536;                       // tokens per selection-mask window
-constexpr int kMaskWords = (int)(2 * kWin / 32);      // all levels of a window (p >= 2)
-
-namespace cg = cooperative_groups;
+constexpr int kOrderThreads = 256;
+constexpr int kOrderItems = 4;                        // tokens per thread
+constexpr int kOrderTile = kOrderThreads * kOrderItems;
 
 __device__ __forceinline__ unsigned long long entry_key(const float* qk, const float* kq,
                                                         int64_t f) {
@@ -90,96 +62,181 @@ __device__ __forceinline__ unsigned long long entry_key(const float* qk, const f
          (unsigned long long)(0xffffffffu - (uint32_t)f);
 }
 
-typedef cub::BlockScan<long long, kSelThreads> ScanLL;
-typedef cub::BlockScan<int, kSelThreads> ScanI;
-typedef cub::BlockReduce<long long, kSelThreads> RedLL;
-
-struct SelSmem {
-  unsigned hist[kBins];
-  unsigned red[kBins];         // this CTA's slice of the cluster-summed histogram
-  uint32_t mask[kMaskWords];   // selection bits of a window, level after level
-  SelState st;                 // the leader's current state (read by the cluster)
-  long long cnt;               // this CTA's selected-entry count
-  long long base;              // its first slot
-  union {
-    typename ScanLL::TempStorage scan_ll;
-    typename ScanI::TempStorage scan_i;
-    typename RedLL::TempStorage red_ll;
-  } tmp;
-};
-
-// Add the digits of the keys f in [lo, hi) that match `prefix` above this
-// pass's digit to h (warp-aggregated shared-memory atomics).  Called by the
-// whole block; every thread runs the same rounds.  kUnroll keys per thread
-// are loaded before any is counted, so their loads overlap.
-__device__ __forceinline__ void count_digits(const float* q, const float* k, int64_t lo,
-                                             int64_t hi, unsigned long long prefix, int pass,
-                                             unsigned* h) {
+__global__ void __launch_bounds__(256) k_sel_hist(LhDims D, const float* __restrict__ qk,
+                                                  const float* __restrict__ kq,
+                                                  unsigned* __restrict__ hist,
+                                                  const SelState* __restrict__ state, int pass) {
+  const int64_t bs = blockIdx.y;                // (b, h) x segment
+  const int64_t bh = bs / D.nseg;
+  const int seg = (int)(bs - bh * D.nseg);
+  unsigned long long prefix = 0;
+  if (pass > 0) {
+    const SelState s = state[bs];
+    if (s.done) return;
+    prefix = s.prefix;
+  }
+  __shared__ unsigned h[kBins];
+  for (int i = threadIdx.x; i < kBins; i += blockDim.x) h[i] = 0;
+  __syncthreads();
   const int shift = c_shift[pass];
-  const int top = shift + c_width[pass];
+  const int hi = shift + c_width[pass];
   const unsigned mask = (1u << c_width[pass]) - 1u;
-  const int64_t span = hi > lo ? hi - lo : 0;
-  const int64_t per = (int64_t)blockDim.x * kUnroll;
-  for (int64_t r0 = 0; r0 < span; r0 += per) {
-    unsigned long long key[kUnroll];
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int64_t f = lo + r0 + (int64_t)u * blockDim.x + threadIdx.x;
-      key[u] = f < hi ? entry_key(q, k, f) : 0ull;
+  const float* q = qk + bh * D.P;
+  const float* k = kq + bh * D.P;
+  const int64_t seg_end = D.seg_lo[seg] + D.seg_len[seg];
+  const int64_t per_block = (D.seg_len[seg] + gridDim.x - 1) / gridDim.x;
+  const int64_t lo = D.seg_lo[seg] + (int64_t)blockIdx.x * per_block;
+  const int64_t end = min(lo + per_block, seg_end);
+  const int64_t span = end > lo ? end - lo : 0;
+  const int64_t rounds = (span + blockDim.x - 1) / blockDim.x;
+  for (int64_t r = 0; r < rounds; ++r) {
+    const int64_t f = lo + r * blockDim.x + threadIdx.x;
+    bool in = f < end;
+    unsigned digit = 0;
+    if (in) {
+      const unsigned long long key = entry_key(q, k, f);
+      in = (hi >= 64) || ((key >> hi) == (prefix >> hi));
+      digit = (unsigned)(key >> shift) & mask;
     }
+    // warp-aggregated increment: one shared atomic per distinct digit
+    const unsigned act = __ballot_sync(0xffffffffu, in);
+    if (in) {
+      const unsigned peers = __match_any_sync(act, digit);
+      if ((threadIdx.x & 31) == (unsigned)(__ffs(peers) - 1)) atomicAdd(&h[digit], __popc(peers));
+    }
+  }
+  __syncthreads();
+  unsigned* g = hist + (bs * kPasses + pass) * kBins;
+  for (int i = threadIdx.x; i < kBins; i += blockDim.x)
+    if (h[i]) atomicAdd(&g[i], h[i]);
+}
+
+// One block of 256 threads per (b, h) and segment; thread t owns digits
+// 2047-8t .. 2040-8t.
+__global__ void __launch_bounds__(256) k_sel_find(LhDims D, const unsigned* __restrict__ hist,
+                                                  SelState* __restrict__ state, int pass) {
+  const int64_t bh = blockIdx.x;                 // (b, h) x segment
+  SelState s;
+  if (pass == 0) {
+    s.prefix = 0;
+    s.need = D.seg_need;
+    s.done = D.seg_need == 0;
+    s.pad = 0;
+    if (s.done) s.prefix = ~0ull;  // nothing is selected
+  } else {
+    s = state[bh];
+  }
+  __syncthreads();
+  if (s.done) {
+    if (pass == 0 && threadIdx.x == 0) state[bh] = s;
+    return;
+  }
+  const unsigned* g = hist + (bh * kPasses + pass) * kBins;
+  unsigned c[8];
+  long long mine = 0;
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int64_t f = lo + r0 + (int64_t)u * blockDim.x + threadIdx.x;
-      const bool in = f < hi && ((top >= 64) || ((key[u] >> top) == (prefix >> top)));
-      const unsigned digit = (unsigned)(key[u] >> shift) & mask;
+  for (int i = 0; i < 8; ++i) {
+    c[i] = g[kBins - 1 - (threadIdx.x * 8 + i)];
+    mine += c[i];
+  }
+  typedef cub::BlockScan<long long, 256> Scan;
+  __shared__ typename Scan::TempStorage tmp;
+  long long before;
+  Scan(tmp).ExclusiveSum(mine, before);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (before < s.need && s.need <= before + (long long)c[i]) {
+      const unsigned digit = kBins - 1 - (threadIdx.x * 8 + i);
+      SelState o;
+      o.prefix = s.prefix | ((unsigned long long)digit << c_shift[pass]);
+      o.need = s.need - before;
+      o.done = (o.need == (long long)c[i]) ? 1 : 0;
+      o.pad = 0;
+      state[bh] = o;
+      if (!o.done && pass == kPasses - 1) lh_report(D.status, LH_ERR_DEVICE_BOUNDS, 100);
+    }
+    before += c[i];
+  }
+}
+
+// Stratified selection: one block of 256 threads per (b, h) and chunk finds
+// the chunk's m-th largest key by the same 11-bit radix passes, reading the
+// chunk's keys once per pass (they stay in L1/L2) and counting digits in
+// shared memory; it stops as soon as every key left in the chosen digit is
+// needed.  state[bs].prefix is then the threshold: selected(f) <=> key(f) >=
+// prefix, and exactly m keys of the chunk pass it (keys are unique).
+__global__ void __launch_bounds__(256) k_sel_chunk(LhDims D, const float* __restrict__ qk,
+                                                   const float* __restrict__ kq,
+                                                   SelState* __restrict__ state) {
+  const int64_t bs = blockIdx.x;                 // (b, h) x chunk
+  const int64_t bh = bs / D.nseg;
+  const int64_t s = bs - bh * D.nseg;
+  const int64_t lo = s * D.n_cand / D.nseg;
+  const int64_t hi_f = (s + 1) * D.n_cand / D.nseg;
+  const float* q = qk + bh * D.P;
+  const float* k = kq + bh * D.P;
+  __shared__ unsigned h[kBins];
+  __shared__ SelState sh;
+  typedef cub::BlockScan<long long, 256> Scan;
+  __shared__ typename Scan::TempStorage tmp;
+  SelState st;
+  st.prefix = 0;
+  st.need = D.seg_need;
+  st.done = 0;
+  st.pad = 0;
+  for (int pass = 0; pass < kPasses; ++pass) {
+    for (int i = threadIdx.x; i < kBins; i += blockDim.x) h[i] = 0;
+    __syncthreads();
+    const int shift = c_shift[pass];
+    const int hi = shift + c_width[pass];
+    const unsigned mask = (1u << c_width[pass]) - 1u;
+    for (int64_t f0 = lo; f0 < hi_f; f0 += blockDim.x) {
+      const int64_t f = f0 + threadIdx.x;
+      bool in = f < hi_f;
+      unsigned digit = 0;
+      if (in) {
+        const unsigned long long key = entry_key(q, k, f);
+        in = (hi >= 64) || ((key >> hi) == (st.prefix >> hi));
+        digit = (unsigned)(key >> shift) & mask;
+      }
       const unsigned act = __ballot_sync(0xffffffffu, in);
       if (in) {
         const unsigned peers = __match_any_sync(act, digit);
         if ((threadIdx.x & 31) == (unsigned)(__ffs(peers) - 1)) atomicAdd(&h[digit], __popc(peers));
       }
     }
-  }
-}
-
-// The digit of this pass that holds the need-th largest key, from the
-// per-digit counts count(d) (thread t owns digits 2047 - kBinsPer t
-// downwards).  The new state goes to *out, written by the one thread whose
-// digit it is.  Whole block.
-template <typename Count>
-__device__ __forceinline__ void find_digit(const SelState& s, int pass, Count count,
-                                           SelState* out, typename ScanLL::TempStorage& tmp) {
-  unsigned c[kBinsPer];
-  long long mine = 0;
+    __syncthreads();
+    unsigned c[8];
+    long long mine = 0;
 #pragma unroll
-  for (int i = 0; i < kBinsPer; ++i) {
-    c[i] = count(kBins - 1 - (threadIdx.x * kBinsPer + i));
-    mine += c[i];
-  }
-  long long before;
-  ScanLL(tmp).ExclusiveSum(mine, before);
-#pragma unroll
-  for (int i = 0; i < kBinsPer; ++i) {
-    if (before < s.need && s.need <= before + (long long)c[i]) {
-      const unsigned digit = kBins - 1 - (threadIdx.x * kBinsPer + i);
-      SelState o;
-      o.prefix = s.prefix | ((unsigned long long)digit << c_shift[pass]);
-      o.need = s.need - before;
-      o.done = (o.need == (long long)c[i]) ? 1 : 0;
-      o.pad = 0;
-      *out = o;
+    for (int i = 0; i < 8; ++i) {
+      c[i] = h[kBins - 1 - (threadIdx.x * 8 + i)];
+      mine += c[i];
     }
-    before += c[i];
+    long long before;
+    Scan(tmp).ExclusiveSum(mine, before);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (before < st.need && st.need <= before + (long long)c[i]) {
+        const unsigned digit = kBins - 1 - (threadIdx.x * 8 + i);
+        SelState o;
+        o.prefix = st.prefix | ((unsigned long long)digit << c_shift[pass]);
+        o.need = st.need - before;
+        o.done = (o.need == (long long)c[i]) ? 1 : 0;
+        o.pad = 0;
+        sh = o;
+      }
+      before += c[i];
+    }
+    __syncthreads();   // sh written by exactly one thread (need <= keys left)
+    st = sh;
+    __syncthreads();   // everyone has read sh and h before the next pass clears h
+    if (st.done) break;
   }
-}
-
-__device__ __forceinline__ SelState start_state(int64_t need) {
-  SelState s;
-  s.prefix = 0;
-  s.need = need;
-  s.done = need == 0;
-  s.pad = 0;
-  if (s.done) s.prefix = ~0ull;   // nothing is selected
-  return s;
+  if (threadIdx.x == 0) {
+    if (!st.done) lh_report(D.status, LH_ERR_DEVICE_BOUNDS, 103);
+    state[bs] = st;
+  }
 }
 
 // thr: the (b, h)'s segment states; an entry of level l < L-1 is compared with
@@ -192,253 +249,160 @@ __device__ __forceinline__ bool selected_entry(const LhDims& D, const float* q, 
   int64_t seg = 0;
   if (D.select_mode == 2) seg = ((f + 1) * D.nseg - 1) / D.n_cand;
   else if (D.nseg > 1) seg = l;
-  return entry_key(q, k, f) >= __ldcg(&thr[seg].prefix);
+  return entry_key(q, k, f) >= thr[seg].prefix;
 }
 
-// Selection bits of the entries that end in tokens [w0, w1) (multiples of
-// the coarsest span), level after level: level l's entries
-// [w0 / p^l, w1 / p^l) at bit offsets moff[l] + j.  Returns this thread's
-// count of set bits.  Whole block; warps take 32-entry words, kUnroll/2
-// words in flight.
-__device__ __forceinline__ int build_masks(const LhDims& D, const float* q, const float* k,
-                                           const SelState* thr, int64_t w0, int64_t w1,
-                                           uint32_t* mask, const int* moff) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int W = kUnroll / 2;
+// Number of selected entries that end on token t.
+__device__ __forceinline__ int count_at(const LhDims& D, const float* q, const float* k,
+                                        const SelState* thr, int64_t t) {
   int n = 0;
+  const uint32_t t1 = (uint32_t)(t + 1);  // N < 2^31
   for (int l = 0; l < D.L; ++l) {
-    const int64_t sp = D.lvl_span[l];
-    const int64_t e0 = w0 / sp, ne = (w1 - w0) / sp;
-    const int words = (int)((ne + 31) / 32);
-    uint32_t* m = mask + moff[l] / 32;
-    for (int wb = warp * W; wb < words; wb += kWarps * W) {
-      bool sel[W];
-#pragma unroll
-      for (int u = 0; u < W; ++u) {
-        const int64_t j = (int64_t)(wb + u) * 32 + lane;
-        sel[u] = (wb + u) < words && j < ne &&
-                 selected_entry(D, q, k, thr, l, D.lvl_off[l] + e0 + j);
-      }
-#pragma unroll
-      for (int u = 0; u < W; ++u) {
-        const uint32_t b = __ballot_sync(0xffffffffu, sel[u]);
-        if (lane == 0 && wb + u < words) {
-          m[wb + u] = b;
-          n += __popc(b);
-        }
-      }
-    }
+    const uint32_t span = (uint32_t)D.lvl_span[l];
+    if (t1 % span) break;  // spans are nested: no coarser level ends here either
+    n += selected_entry(D, q, k, thr, l, D.lvl_off[l] + t1 / span - 1);
   }
   return n;
 }
 
-__device__ __forceinline__ bool mask_bit(const uint32_t* mask, int64_t bit) {
-  return (mask[bit >> 5] >> (bit & 31)) & 1u;
-}
-
-// One cluster of CL CTAs per (b, h) (blockIdx.y); see the file comment.
-template <int CL>
-__global__ void __launch_bounds__(kSelThreads) k_select(LhDims D, const float* __restrict__ qk,
-                                                        const float* __restrict__ kq,
-                                                        SelState* __restrict__ state,
-                                                        int32_t* __restrict__ sel_idx,
-                                                        int32_t* __restrict__ slot_map) {
-  cg::cluster_group cluster = cg::this_cluster();
-  __shared__ SelSmem sm;
-  const int c = (int)cluster.block_rank();
+__global__ void __launch_bounds__(kOrderThreads) k_order_count(LhDims D, const float* __restrict__ qk,
+                                                              const float* __restrict__ kq,
+                                                              const SelState* __restrict__ state,
+                                                              int* __restrict__ blk_cnt, int nblk) {
   const int64_t bh = blockIdx.y;
+  const SelState* thr = state + bh * D.nseg;
   const float* q = qk + bh * D.P;
   const float* k = kq + bh * D.P;
-  SelState* thr = state + bh * D.nseg;
-  // this CTA's tokens [t0, t1): whole coarsest-level windows
-  const int64_t span_top = D.lvl_span[D.L - 1];
-  const int64_t n_top = D.lvl_size[D.L - 1];
-  const int64_t tc = (n_top + CL - 1) / CL * span_top;
-  const int64_t t0 = min((int64_t)c * tc, D.N), t1 = min(t0 + tc, D.N);
+  const int64_t t0 = (int64_t)blockIdx.x * kOrderTile;
+  int n = 0;
+  for (int i = 0; i < kOrderItems; ++i) {
+    const int64_t t = t0 + (int64_t)i * kOrderThreads + threadIdx.x;
+    if (t < D.N) n += count_at(D, q, k, thr, t);
+  }
+  typedef cub::BlockReduce<int, kOrderThreads> Red;
+  __shared__ typename Red::TempStorage tmp;
+  const int tot = Red(tmp).Sum(n);
+  if (threadIdx.x == 0) blk_cnt[bh * nblk + blockIdx.x] = tot;
+}
 
-  // ---- selection
-  if (D.select_mode == 2) {
-    // chunks s = c, c + CL, ...: one CTA runs all radix passes of a chunk
-    for (int64_t sg = c; sg < D.nseg; sg += CL) {
-      const int64_t lo = sg * D.n_cand / D.nseg, hi = (sg + 1) * D.n_cand / D.nseg;
-      SelState st = start_state(D.seg_need);
-      for (int pass = 0; pass < kPasses && !st.done; ++pass) {
-        for (int i = threadIdx.x; i < kBins; i += blockDim.x) sm.hist[i] = 0;
-        __syncthreads();
-        count_digits(q, k, lo, hi, st.prefix, pass, sm.hist);
-        __syncthreads();
-        find_digit(st, pass, [&](int d) { return sm.hist[d]; }, &sm.st, sm.tmp.scan_ll);
-        __syncthreads();                // sm.st written by exactly one thread
-        st = sm.st;
-        __syncthreads();                // read before the next pass clears hist
-      }
-      if (threadIdx.x == 0) {
-        if (!st.done) lh_report(D.status, LH_ERR_DEVICE_BOUNDS, 103);
-        thr[sg] = st;
-      }
-    }
-  } else {
-    constexpr int kSlice = kBins / CL;  // digits whose cluster sum this CTA forms
-    for (int sg = 0; sg < D.nseg; ++sg) {
-      // levels of this segment: all finer ones (mode 0) or level sg (mode 1)
-      const int l_lo = D.nseg > 1 ? sg : 0;
-      const int l_hi = D.nseg > 1 ? sg + 1 : D.L - 1;
-      SelState st = start_state(D.seg_need);
-      for (int pass = 0; pass < kPasses && !st.done; ++pass) {
-        for (int i = threadIdx.x; i < kBins; i += blockDim.x) sm.hist[i] = 0;
-        __syncthreads();
-        for (int l = l_lo; l < l_hi; ++l) {
-          const int64_t sp = D.lvl_span[l];
-          count_digits(q, k, D.lvl_off[l] + t0 / sp, D.lvl_off[l] + t1 / sp, st.prefix, pass,
-                       sm.hist);
-        }
-        cluster.sync();                 // every CTA's histogram is complete
-        for (int i = threadIdx.x; i < kSlice; i += blockDim.x) {
-          unsigned tot = 0;
-#pragma unroll
-          for (int r = 0; r < CL; ++r) tot += cluster.map_shared_rank(sm.hist, r)[c * kSlice + i];
-          sm.red[i] = tot;
-        }
-        cluster.sync();                 // the summed histogram lies in the CTAs' slices
-        if (c == 0)
-          find_digit(st, pass, [&](int d) {
-            return cluster.map_shared_rank(sm.red, d / kSlice)[d % kSlice];
-          }, &sm.st, sm.tmp.scan_ll);
-        cluster.sync();                 // the leader's state is published
-        st = *cluster.map_shared_rank(&sm.st, 0);
-      }
-      if (c == 0 && threadIdx.x == 0) {
-        if (!st.done) lh_report(D.status, LH_ERR_DEVICE_BOUNDS, 100);
-        thr[sg] = st;
-      }
-      cluster.sync();                   // every CTA has read the leader's sm.st
-    }
+// One block per (b, h): exclusive scan of the block counts, in place.
+__global__ void __launch_bounds__(1024) k_order_scan(LhDims D, int* __restrict__ blk_cnt, int nblk) {
+  const int64_t bh = blockIdx.x;
+  int* c = blk_cnt + bh * nblk;
+  typedef cub::BlockScan<int, 1024> Scan;
+  __shared__ typename Scan::TempStorage tmp;
+  __shared__ int carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < nblk; base += 1024) {
+    const int i = base + threadIdx.x;
+    const int x = i < nblk ? c[i] : 0;
+    int ex, agg;
+    Scan(tmp).ExclusiveSum(x, ex, agg);
+    if (i < nblk) c[i] = carry + ex;
+    __syncthreads();
+    if (threadIdx.x == 0) carry += agg;
+    __syncthreads();
   }
-  __threadfence();
-  cluster.sync();                       // thresholds in global memory, seen by the cluster
+  if (threadIdx.x == 0 && carry != D.S) lh_report(D.status, LH_ERR_DEVICE_BOUNDS, 101);
+}
 
-  // ---- order.  Bit offsets of each level inside a window's masks.
-  __shared__ int moff[LH_MAX_LEVELS];
-  if (threadIdx.x == 0) {
-    int o = 0;
-    for (int l = 0; l < D.L; ++l) {
-      moff[l] = o;
-      o += (int)(((kWin / D.lvl_span[l]) + 31) / 32) * 32;
-    }
+__global__ void __launch_bounds__(kOrderThreads) k_order_emit(LhDims D, const float* __restrict__ qk,
+                                                             const float* __restrict__ kq,
+                                                             const SelState* __restrict__ state,
+                                                             const int* __restrict__ blk_off, int nblk,
+                                                             int32_t* __restrict__ sel_idx,
+                                                             int32_t* __restrict__ slot_map) {
+  const int64_t bh = blockIdx.y;
+  const SelState* thr = state + bh * D.nseg;
+  const float* q = qk + bh * D.P;
+  const float* k = kq + bh * D.P;
+  // each thread owns kOrderItems consecutive tokens so the scan order is t order
+  const int64_t t0 = (int64_t)blockIdx.x * kOrderTile + (int64_t)threadIdx.x * kOrderItems;
+  int n = 0;
+  for (int i = 0; i < kOrderItems; ++i) {
+    const int64_t t = t0 + i;
+    if (t < D.N) n += count_at(D, q, k, thr, t);
   }
-  __syncthreads();
-  const int64_t win = kWin / span_top * span_top;    // a multiple of the coarsest span
-  const int64_t nwin = (t1 - t0 + win - 1) / win;
-  long long n = 0;
-  for (int64_t w0 = t0; w0 < t1; w0 += win) {
-    n += build_masks(D, q, k, thr, w0, min(w0 + win, t1), sm.mask, moff);
-    __syncthreads();                    // masks rebuilt by the next window
-  }
-  n = RedLL(sm.tmp.red_ll).Sum(n);
-  if (threadIdx.x == 0) sm.cnt = n;
-  cluster.sync();
-  if (threadIdx.x == 0) {
-    long long base = 0, total = 0;
-    for (int r = 0; r < CL; ++r) {
-      const long long x = *cluster.map_shared_rank(&sm.cnt, r);
-      if (r < c) base += x;
-      total += x;
-    }
-    sm.base = base;
-    if (c == 0 && total != D.S) lh_report(D.status, LH_ERR_DEVICE_BOUNDS, 101);
-  }
-  __syncthreads();
+  typedef cub::BlockScan<int, kOrderThreads> Scan;
+  __shared__ typename Scan::TempStorage tmp;
+  int ex;
+  Scan(tmp).ExclusiveSum(n, ex);
+  int slot = blk_off[bh * nblk + blockIdx.x] + ex;
   int32_t* si = sel_idx + bh * D.S;
-  int32_t* smap = slot_map + bh * D.P;
-  long long slot0 = sm.base;
-  for (int64_t w0 = t0; w0 < t1; w0 += win) {
-    const int64_t w1 = min(w0 + win, t1);
-    if (nwin > 1) {                     // one window: its masks are still there
-      build_masks(D, q, k, thr, w0, w1, sm.mask, moff);
-      __syncthreads();
-    }
-    for (int64_t tt = w0; tt < w1; tt += kTile) {
-      const int64_t ta = tt + (int64_t)threadIdx.x * kItems;   // kItems consecutive tokens
-      int cnt = 0;
-#pragma unroll
-      for (int u = 0; u < kItems; ++u) {
-        const int64_t t = ta + u;
-        if (t >= w1) break;
-        const int64_t t1p = t + 1;
-        for (int l = 0; l < D.L; ++l) {
-          const int64_t sp = D.lvl_span[l];
-          if (t1p % sp) break;
-          cnt += mask_bit(sm.mask, moff[l] + (t1p / sp - 1 - w0 / sp));
-        }
+  int32_t* sm = slot_map + bh * D.P;
+  for (int i = 0; i < kOrderItems; ++i) {
+    const int64_t t = t0 + i;
+    if (t >= D.N) break;
+    const uint32_t t1 = (uint32_t)(t + 1);
+    for (int l = 0; l < D.L; ++l) {
+      const uint32_t span = (uint32_t)D.lvl_span[l];
+      if (t1 % span) break;
+      const int64_t f = D.lvl_off[l] + t1 / span - 1;
+      if (selected_entry(D, q, k, thr, l, f)) {
+        if (slot < D.S) si[slot] = (int32_t)f;
+        else lh_report(D.status, LH_ERR_DEVICE_BOUNDS, 102);
+        sm[f] = slot++;
+      } else {
+        sm[f] = -1;
       }
-      int ex, agg;
-      ScanI(sm.tmp.scan_i).ExclusiveSum(cnt, ex, agg);
-      long long slot = slot0 + ex;
-      for (int u = 0; u < kItems; ++u) {
-        const int64_t t = ta + u;
-        if (t >= w1) break;
-        const int64_t t1p = t + 1;
-        for (int l = 0; l < D.L; ++l) {
-          const int64_t sp = D.lvl_span[l];
-          if (t1p % sp) break;
-          const int64_t i = t1p / sp - 1;
-          const int64_t f = D.lvl_off[l] + i;
-          if (mask_bit(sm.mask, moff[l] + (i - w0 / sp))) {
-            if (slot < D.S) si[slot] = (int32_t)f;
-            else lh_report(D.status, LH_ERR_DEVICE_BOUNDS, 102);
-            smap[f] = (int32_t)slot++;
-          } else {
-            smap[f] = -1;
-          }
-        }
-      }
-      slot0 += agg;
-      __syncthreads();                  // scan storage reused by the next tile
     }
   }
-  cluster.sync();                       // no CTA leaves while others read its shared memory
 }
 
-template <int CL>
-cudaError_t launch_select(const LhDims& D, const float* qk, const float* kq, SelState* state,
-                          int32_t* sel_idx, int32_t* slot_map, cudaStream_t st) {
-  if (CL > 8) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(k_select<CL>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(CL, (unsigned)((int64_t)D.B * D.H));
-  cfg.blockDim = dim3(kSelThreads);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = CL;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_select<CL>, D, qk, kq, state, sel_idx, slot_map);
-}
+inline int64_t order_blocks(const LhDims& D) { return (D.N + kOrderTile - 1) / kOrderTile; }
 
 }  // namespace
 
 size_t lh_select_ws_bytes(const LhDims& D) {
-  const int64_t BS = (int64_t)D.B * D.H * D.nseg;
-  return ((size_t)BS * sizeof(SelState) + 255) & ~(size_t)255;   // per-segment thresholds
+  const int64_t BH = (int64_t)D.B * D.H;
+  const int64_t BS = BH * D.nseg;
+  size_t b = 0;
+  if (D.select_mode != 2) b += (size_t)BS * kPasses * kBins * sizeof(unsigned);  // histograms
+  b += (size_t)BS * sizeof(SelState);
+  b = (b + 255) & ~(size_t)255;
+  b += (size_t)BH * order_blocks(D) * sizeof(int);
+  return (b + 255) & ~(size_t)255;
 }
 
 cudaError_t lh_launch_select(const LhDims& D, const float* qk, const float* kq,
                              int32_t* sel_idx, int32_t* slot_map, void* ws, cudaStream_t st,
                              int* launches) {
-  SelState* state = reinterpret_cast<SelState*>(ws);
-  // 16-CTA clusters where the device schedules them, else the portable 8
-  cudaError_t e = launch_select<16>(D, qk, kq, state, sel_idx, slot_map, st);
-  if (e != cudaSuccess) {
-    (void)cudaGetLastError();
-    e = launch_select<8>(D, qk, kq, state, sel_idx, slot_map, st);
+  const int64_t BH = (int64_t)D.B * D.H;
+  const int64_t BS = BH * D.nseg;                 // (b, h) x selection segment
+  const size_t hist_bytes =
+      D.select_mode == 2 ? 0 : (size_t)BS * kPasses * kBins * sizeof(unsigned);
+  unsigned* hist = reinterpret_cast<unsigned*>(ws);
+  SelState* state = reinterpret_cast<SelState*>(reinterpret_cast<char*>(ws) + hist_bytes);
+  size_t off = hist_bytes + (size_t)BS * sizeof(SelState);
+  off = (off + 255) & ~(size_t)255;
+  int* blk = reinterpret_cast<int*>(reinterpret_cast<char*>(ws) + off);
+  const int nblk = (int)order_blocks(D);
+  int n = 0;
+  if (D.select_mode == 2) {
+    k_sel_chunk<<<(unsigned)BS, 256, 0, st>>>(D, qk, kq, state);
+    n += 1;
+  } else if (D.n_cand > 0) {
+    cudaError_t e = cudaMemsetAsync(hist, 0, hist_bytes, st);
+    if (e != cudaSuccess) return e;
+    // ~8 candidates per thread per block keeps every SM busy on one head too
+    int64_t per = (D.seg_len[0] + 148 * 4 - 1) / (148 * 4);   // segment 0 is the largest
+    per = per < 2048 ? 2048 : per;
+    const unsigned gx = (unsigned)((D.seg_len[0] + per - 1) / per);
+    for (int pass = 0; pass < kPasses; ++pass) {
+      k_sel_hist<<<dim3(gx, (unsigned)BS), 256, 0, st>>>(D, qk, kq, hist, state, pass);
+      k_sel_find<<<(unsigned)BS, 256, 0, st>>>(D, hist, state, pass);
+      n += 2;
+    }
+  } else {
+    k_sel_find<<<(unsigned)BS, 256, 0, st>>>(D, hist, state, 0);   // reads no histogram
+    n += 1;
   }
-  if (launches) *launches = 1;
-  return e != cudaSuccess ? e : cudaGetLastError();
+  k_order_count<<<dim3(nblk, (unsigned)BH), kOrderThreads, 0, st>>>(D, qk, kq, state, blk, nblk);
+  k_order_scan<<<(unsigned)BH, 1024, 0, st>>>(D, blk, nblk);
+  k_order_emit<<<dim3(nblk, (unsigned)BH), kOrderThreads, 0, st>>>(D, qk, kq, state, blk, nblk,
+                                                                   sel_idx, slot_map);
+  n += 3;
+  if (launches) *launches = n;
+  return cudaGetLastError();
 }

@@ -87,8 +87,7 @@ typedef struct {
 } lh_config;
 
 /* Returns LH_OK when the config is valid and supported: B, N, H >= 1,
- * p >= 2, 1 <= L <= 6, p^(L-1) | N, p^(L-1) <= 65536 (else
- * LH_ERR_UNSUPPORTED), 0 <= (L-1) p k <= sum_{l<L-1} N/p^l,
+ * p >= 2, 1 <= L <= 6, p^(L-1) | N, 0 <= (L-1) p k <= sum_{l<L-1} N/p^l,
  * d in {64, 128}, every index fits in int32 per (b, h), and B H (times L-1
  * in select_mode 1) <= 65535, the launch-grid limit of the per-head
  * selection kernels (else LH_ERR_UNSUPPORTED). */
@@ -165,11 +164,11 @@ lh_status lh_score_topk(const lh_config* cfg, const float* qk, const float* kq,
  *  - Same arguments and results as lh_score_topk, minus ws / ws_bytes.
  *  - Returns LH_ERR_WORKSPACE, before any launch, when the selection
  *    scratch of cfg (the part of fwd_ws that lh_score_topk uses) exceeds the
- *    array.  That scratch is one 24-byte threshold per selection segment:
- *    B*H*24 bytes in select_mode 0, B*H*(L-1)*24 in mode 1 and B*H*n*24 for
- *    the n chunks of mode 2 (rounded up to 256 bytes).  So every config of
- *    modes 0 and 1 that lh_config_check accepts fits, and mode 2 fits up to
- *    B*H*n = 349525 chunks.
+ *    array.  That scratch is, roughly: select_mode 0, B*H*48 KB of digit
+ *    histograms; select_mode 1, B*H*(L-1)*48 KB; select_mode 2, B*H*n*24
+ *    bytes for its n chunks; plus B*H*N/256 bytes of order counts in every
+ *    mode.  So B*H <= 128 heads fit at N = 2^20 in modes 0 and 2, and
+ *    B*H*(L-1) <= 128 in mode 1.
  *  - The first call on a device looks up the array's device address (once
  *    per device, with that device current); make that first call before any
  *    stream capture.

@@ -67,9 +67,10 @@ def test_noalloc_topk_rejects_shapes_beyond_its_array():
 
     x = torch.empty(16, dtype=torch.float32, device="cuda")
     i = torch.empty(16, dtype=torch.int32, device="cuda")
-    # stratified selection with 512 heads of 1024 chunks: 24 bytes of
-    # threshold per chunk, 12 MiB in all
-    for cfg in (L.make_config(64, 1 << 20, 8, 128, 3, 4, 1024, select_mode=2, select_chunk=8),):
+    # B*H = 512 heads: ~27 MB of scratch; and the per-level quota at B*H = 128,
+    # L = 3, N = 2^20, whose two segments per head need ~13 MB
+    for cfg in (L.make_config(64, 1 << 20, 8, 128, 3, 4, 1024),
+                L.make_config(16, 1 << 20, 8, 128, 3, 4, 1024, select_mode=1)):
         with pytest.raises(L.LighthouseError) as e:
             L.lh_score_topk_noalloc(cfg, x, x, i, i)
         assert e.value.code == 3  # LH_ERR_WORKSPACE, raised before any launch
