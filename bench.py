@@ -176,7 +176,9 @@ def bench_config(args, w, ws):
     return {"workload": f"{w['name']}: B={B} N={N} H={H} d={d} L={Lv} p={p} k={k} S={S}",
             "step": "lh_forward + lh_backward stages (fwd+bwd)",
             "l2": f"inputs larger than L2 ({tok_gib:.2f} GiB of Q,K,V per step); no flush",
-            "parallelism": f"replicas x{ws} (independent layers, no collective)",
+            "parallelism": (f"head split over {ws} ranks (one layer; no collective)"
+                            if args.head_split and ws > 1 else
+                            f"replicas x{ws} (independent layers, no collective)"),
             "selection": SELECT_NAMES[args.select_mode] +
             (f", {args.select_chunk} per chunk" if args.select_mode == 2 else "")}
 
@@ -188,6 +190,15 @@ def run_ours(args, w, ws, rank, local):
     dev = torch.device("cuda", local)
     qh, kh, vh = make_qkv(B, N, H, d, seed=args.workload)
     doh = make_dout(B, N, H, d, seed=args.workload)
+    # head split: this rank runs the whole layer on its contiguous head range
+    # of the one job-wide layer (the job's tokens are counted once)
+    share, w_job = ws, w
+    if args.head_split and ws > 1:
+        from hierarchical_selection_attention_b200.heads import head_range
+        h0, h1 = head_range(H, ws, rank)
+        qh, kh, vh, doh = (x[:, :, h0:h1].contiguous() for x in (qh, kh, vh, doh))
+        H, share = h1 - h0, 1
+        w = dict(w, H=H)
     q, kk, v, dout = (t.to(dev) for t in (qh, kh, vh, doh))
     sel = dict(select_mode=args.select_mode, select_chunk=args.select_chunk)
     cfg = L.make_config(B, N, H, d, Lv, p, k, **sel)
@@ -311,7 +322,7 @@ def run_ours(args, w, ws, rank, local):
         L.check_device_status()
         e2e_ms = max_over_ranks(a.elapsed_time(b), ws) / n_e2e
         nbytes = B * N * H * d * 2
-        e2e = {"value": ws * B * N / (e2e_ms / 1e3), "unit": UNIT, "ms_per_step": e2e_ms,
+        e2e = {"value": share * B * N / (e2e_ms / 1e3), "unit": UNIT, "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": 4 * nbytes, "d2h_bytes_per_step": 4 * nbytes,
                "api": "LighthouseLayer.forward/backward (lh_forward + lh_backward), pinned host buffers; upload, compute and download on three streams, overlapped across steps"}
 
@@ -350,12 +361,14 @@ def run_ours(args, w, ws, rank, local):
     launches = args.steps * (L.lh_forward_launches(cfg) + L.lh_backward_launches(cfg))
     ms_step = total_ms / args.steps
     line = {
-        "metric": METRIC, "value": job_tokens_per_s(ws, B, N, ms_step), "unit": UNIT, "n_gpus": ws,
+        "metric": METRIC, "value": job_tokens_per_s(share, B, N, ms_step), "unit": UNIT, "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "strong" if share == 1 and ws > 1 else "weak",
+        "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded: N(0,1) x per-token lognormal(0,0.5), 64 heavy tokens x4)",
-        "config": bench_config(args, w, ws),
-        "fwd_tokens_per_s": ws * B * N / (fwd_ms / 1e3), "fwd_ms": fwd_ms,
+        "config": bench_config(args, w_job, ws),
+        "heads_this_rank": H,
+        "fwd_tokens_per_s": share * B * N / (fwd_ms / 1e3), "fwd_ms": fwd_ms,
         "stages": per_stage, "roofline": roof, "e2e": e2e, "gpu_launches": launches,
         "clocks": clocks,
     }
@@ -672,6 +685,9 @@ def main():
                     help="selection: 0 joint top-k (default), 1 per-level quota, 2 stratified")
     ap.add_argument("--select-chunk", type=int, default=0,
                     help="per-chunk quota m of the stratified selection")
+    ap.add_argument("--head-split", action="store_true",
+                    help="N > 1: split one layer's heads over the ranks (strong scaling) "
+                         "instead of running N replicas (weak scaling)")
     ap.add_argument("--ring", type=int, default=0,
                     help="time the context-parallel layer with this many shards on one GPU")
     ap.add_argument("--full-layer", action="store_true",
@@ -696,6 +712,8 @@ def main():
         return
 
     ws, rank, local = dist_init()
+    if ws != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but {ws} ranks were launched")
     try:
         line = run_ours(args, w, ws, rank, local)
         if rank == 0:

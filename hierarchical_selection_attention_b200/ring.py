@@ -181,7 +181,7 @@ class LighthouseRingLayer:
     contiguous view; for B > 1 it is copied out and back."""
 
     def __init__(self, B, N, H, d, L, p, k, R, scale: float = 0.0, device="cuda",
-                 select_mode: int = 0, select_chunk: int = 0):
+                 select_mode: int = 0, select_chunk: int = 0, scatter_mode: int = 0):
         import torch
         from hierarchical_selection_attention_b200 import lighthouse as lh
         if R < 1 or N % R:
@@ -189,7 +189,8 @@ class LighthouseRingLayer:
         self.lh, self.torch = lh, torch
         self.B, self.N, self.H, self.d, self.R, self.Ns = B, N, H, d, R, N // R
         self.shards = [lh.LighthouseLayer(B, self.Ns, H, d, L, p, k, scale, device=device,
-                                          select_mode=select_mode, select_chunk=select_chunk)
+                                          select_mode=select_mode, select_chunk=select_chunk,
+                                          scatter_mode=scatter_mode)
                        for _ in range(R)]
         self.cfg = self.shards[0].cfg
         self.S = self.shards[0].S

@@ -125,3 +125,43 @@ def test_ring_layer_is_deterministic(lib):
     assert torch.equal(oa, ob)
     for a, b in zip(ga, gb):
         assert torch.equal(a, b)
+
+
+# the other selection readings and the integer-atomic scatter, shard by shard
+@pytest.mark.parametrize("mode,chunk,scatter", [(1, 0, 0), (2, 16, 0), (0, 0, 1)])
+def test_ring_layer_other_modes(lib, mode, chunk, scatter):
+    L, ring = lib
+    B, N, H, d, Lv, p, k, R = 1, 8192, 2, 64, 3, 4, 32, 2
+    qh, kh, vh = make_qkv(B, N, H, d, seed=9)
+    doh = make_dout(B, N, H, d, seed=9)
+    q, kk, v, dout = (t.cuda() for t in (qh, kh, vh, doh))
+    layer = ring.LighthouseRingLayer(B, N, H, d, Lv, p, k, R, select_mode=mode, select_chunk=chunk,
+                                     scatter_mode=scatter)
+    o = layer.forward(q, kk, v)
+    dq, dk, dv = layer.backward(dout)
+    torch.cuda.synchronize()
+    L.check_device_status()
+    Ns = N // R
+    for h in range(H):
+        tag = f"R={R} mode={mode} scatter={scatter} [h={h}]"
+        qx, kx, vx, dox = (head(x, 0, h) for x in (qh, kh, vh, doh))
+        st = lo.cp_forward_head(qx, kx, vx, Lv, p, k, R, parity=True, select_mode=mode,
+                                select_chunk=chunk)
+        for r, sh in enumerate(st["shards"]):
+            sv = layer.shards[r].views()
+            np.testing.assert_array_equal(sv["sel_idx"][0, h].cpu().numpy(), sh["sel_idx"])
+        dog = np.concatenate([lo.round_bf16(lo.scatter_bwd(dox[r * Ns:(r + 1) * Ns], sh["sel_idx"],
+                                                           Ns, Lv, p))
+                              for r, sh in enumerate(st["shards"])])
+        eo, eq, ek, ev = attn_envelopes_full(st["qg"], st["kg"], st["vg"], dog, st["scale"])
+        Sr = layer.S
+        env_o = np.concatenate([lo.scatter(eo[r * Sr:(r + 1) * Sr], sh["slot_map"], Ns, Lv, p)
+                                for r, sh in enumerate(st["shards"])])
+        assert_close(o[0, :, h, :].double().cpu().numpy(), st["o"], f"ring O {tag}", env=env_o)
+        want = lo.cp_backward_head(st, dox)
+        for name, gpu, w, env in (("dQ", dq, want[0], eq), ("dK", dk, want[1], ek),
+                                  ("dV", dv, want[2], ev)):
+            env_t = np.concatenate([lo.pyramid_bwd(env[r * Sr:(r + 1) * Sr], sh["slot_map"], Ns,
+                                                   Lv, p)
+                                    for r, sh in enumerate(st["shards"])])
+            assert_close(gpu[0, :, h, :].double().cpu().numpy(), w, f"ring {name} {tag}", env=env_t)
