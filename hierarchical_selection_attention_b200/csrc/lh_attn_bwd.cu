@@ -33,6 +33,8 @@
 // several steps reach are summed in fp32 accumulators (`first` writes them
 // without reading, `last` writes the bf16 result instead), in step order,
 // so the sums stay bitwise reproducible.
+#include <type_traits>
+
 #include "lh_sm100.cuh"
 
 namespace {
@@ -307,27 +309,33 @@ __global__ void __launch_bounds__(kThreadsDkdv, 1)
       tmem_ld32(cS, *reinterpret_cast<uint32_t(*)[32]>(&p[0]));
       tmem_ld32(cS + 32, *reinterpret_cast<uint32_t(*)[32]>(&p[32]));
       tmem_ld_wait();
+      // two copies of the loop, so that off-diagonal tiles carry no
+      // per-column compare
+      auto p_tile = [&](auto masked) {
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t pk[8];
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t pk[8];
 #pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          const int j = ch * 16 + e;
-          const float2 x = f2_unpack(f2_mul(f2_pack(__uint_as_float(p[j]), __uint_as_float(p[j + 1])), c2));
-          float p0 = ex2(x.x);
-          float p1 = ex2(x.y);
-          if (diag) {
-            p0 = (qc0 + j >= kvrow) ? p0 : 0.f;
-            p1 = (qc0 + j + 1 >= kvrow) ? p1 : 0.f;
+          for (int e = 0; e < 16; e += 2) {
+            const int j = ch * 16 + e;
+            const float2 x = f2_unpack(f2_mul(f2_pack(__uint_as_float(p[j]), __uint_as_float(p[j + 1])), c2));
+            float p0 = ex2(x.x);
+            float p1 = ex2(x.y);
+            if constexpr (decltype(masked)::value) {
+              p0 = (qc0 + j >= kvrow) ? p0 : 0.f;
+              p1 = (qc0 + j + 1 >= kvrow) ? p1 : 0.f;
+            }
+            p[j] = __float_as_uint(p0);
+            p[j + 1] = __float_as_uint(p1);
+            pk[e >> 1] = pack_bf16x2(p0, p1);
           }
-          p[j] = __float_as_uint(p0);
-          p[j + 1] = __float_as_uint(p1);
-          pk[e >> 1] = pack_bf16x2(p0, p1);
+          // packed P of columns 16 ch .. 16 ch + 15 lands on fp32 columns
+          // 8 ch .. 8 ch + 7 of this thread's range, already read above
+          tmem_st8(cS + ch * 8, pk);
         }
-        // packed P of columns 16 ch .. 16 ch + 15 lands on fp32 columns
-        // 8 ch .. 8 ch + 7 of this thread's range, already read above
-        tmem_st8(cS + ch * 8, pk);
-      }
+      };
+      if (diag) p_tile(std::true_type{});
+      else p_tile(std::false_type{});
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bars->pready);
@@ -592,17 +600,21 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
       tc_fence_before();
       mbar_arrive(&bars->sfree[sb]);
       const uint64_t c2 = f2_pack(c, c), nl2 = f2_pack(-lrow, -lrow);
+      auto p_row = [&](auto masked) {   // two copies: no compare off the diagonal
 #pragma unroll
-      for (int e = 0; e < 64; e += 2) {
-        const float2 x = f2_unpack(f2_fma(f2_pack(__uint_as_float(p[e]), __uint_as_float(p[e + 1])), c2, nl2));
-        float p0 = ex2(x.x), p1 = ex2(x.y);
-        if (diag) {
-          p0 = (kc0 + e <= qrow) ? p0 : 0.f;
-          p1 = (kc0 + e + 1 <= qrow) ? p1 : 0.f;
+        for (int e = 0; e < 64; e += 2) {
+          const float2 x = f2_unpack(f2_fma(f2_pack(__uint_as_float(p[e]), __uint_as_float(p[e + 1])), c2, nl2));
+          float p0 = ex2(x.x), p1 = ex2(x.y);
+          if constexpr (decltype(masked)::value) {
+            p0 = (kc0 + e <= qrow) ? p0 : 0.f;
+            p1 = (kc0 + e + 1 <= qrow) ? p1 : 0.f;
+          }
+          p[e] = __float_as_uint(p0);
+          p[e + 1] = __float_as_uint(p1);
         }
-        p[e] = __float_as_uint(p0);
-        p[e + 1] = __float_as_uint(p1);
-      }
+      };
+      if (diag) p_row(std::true_type{});
+      else p_row(std::false_type{});
 #pragma unroll
       for (int g = 0; g < 4; ++g) materialize16(p + 16 * g);
       // ---- dS = P (dP - D), bf16 into TMEM; the dP loads run one chunk ahead

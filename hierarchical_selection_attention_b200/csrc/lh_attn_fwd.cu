@@ -42,6 +42,8 @@
 // plain single-block attention.
 #include <cudaTypedefs.h>
 
+#include <type_traits>
+
 #include "lh_sm100.cuh"
 
 namespace {
@@ -248,25 +250,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint64_t rs2[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) rs2[u] = f2_pack(0.f, 0.f);
+      // two copies of the loop, so that unmasked tiles (all but one) carry no
+      // per-column compare
+      auto exp_tile = [&](auto masked) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[8];
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[8];
 #pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          const int i = c * 16 + e;
-          const float2 x = f2_unpack(f2_fma(f2_pack(__uint_as_float(s[i]), __uint_as_float(s[i + 1])), sc2, nm2));
-          float p0 = ex2(x.x), p1 = ex2(x.y);
-          if (msk) {
-            p0 = (c0 + i < lim) ? p0 : 0.f;
-            p1 = (c0 + i + 1 < lim) ? p1 : 0.f;
+          for (int e = 0; e < 16; e += 2) {
+            const int i = c * 16 + e;
+            const float2 x = f2_unpack(f2_fma(f2_pack(__uint_as_float(s[i]), __uint_as_float(s[i + 1])), sc2, nm2));
+            float p0 = ex2(x.x), p1 = ex2(x.y);
+            if constexpr (decltype(masked)::value) {
+              p0 = (c0 + i < lim) ? p0 : 0.f;
+              p1 = (c0 + i + 1 < lim) ? p1 : 0.f;
+            }
+            rs2[(i >> 1) & 3] = f2_add(rs2[(i >> 1) & 3], f2_pack(p0, p1));
+            pk[e >> 1] = pack_bf16x2(p0, p1);
           }
-          rs2[(i >> 1) & 3] = f2_add(rs2[(i >> 1) & 3], f2_pack(p0, p1));
-          pk[e >> 1] = pack_bf16x2(p0, p1);
+          // P of columns 16 c .. 16 c + 15 of this half lands on columns
+          // 8 c .. 8 c + 7, whose scores were read above
+          tmem_st8(tS + c * 8, pk);
         }
-        // P of columns 16 c .. 16 c + 15 of this half lands on columns
-        // 8 c .. 8 c + 7, whose scores were read above
-        tmem_st8(tS + c * 8, pk);
-      }
+      };
+      if (msk) exp_tile(std::true_type{});
+      else exp_tile(std::false_type{});
       const float2 ra = f2_unpack(f2_add(rs2[0], rs2[1])), rb = f2_unpack(f2_add(rs2[2], rs2[3]));
       const float rs = (ra.x + ra.y) + (rb.x + rb.y);
       lsum = lsum * alpha + rs;
