@@ -354,7 +354,7 @@ def run_ours(args, w, ws, rank, local):
         roof = {"bound": "tensor", "kernel": dom, "achieved": round(ach, 1), "peak": pk["tf_sust"],
                 "unit": "TFLOP/s", "frac": round(ach / pk["tf_sust"], 4), "traffic": None}
     roof["peak_source"] = f"{pk['src']} (bf16 sustained for tensor, copy for HBM)"
-    traffic = load_traffic(dom)
+    traffic = load_traffic(dom, w_job["name"])
     if traffic is not None:
         roof["traffic"] = traffic
 
@@ -375,15 +375,17 @@ def run_ours(args, w, ws, rank, local):
     return line
 
 
-def load_traffic(kernel):
+def load_traffic(kernel, workload):
     """Per-launch DRAM bytes of the dominant kernel from the committed ncu
-    summary (profiles/traffic.json), if it was captured for this kernel."""
+    summary (profiles/traffic.json), if it was captured for this kernel on
+    this workload (null otherwise: the bytes do not carry over)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    j = json.load(open(p))
-    ent = j.get(kernel)
-    return None if ent is None else ent.get("dram_bytes_per_launch")
+    ent = json.load(open(p)).get(kernel)
+    if ent is None or ent.get("workload_name") != workload:
+        return None
+    return ent.get("dram_bytes_per_launch")
 
 
 # ----------------------------------------------------------- oracle timing --
