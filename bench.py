@@ -79,6 +79,41 @@ def algorithmic(w):
     }
 
 
+def algorithmic_writes(w):
+    """The part of each HBM stage's algorithmic bytes that is written."""
+    B, N, H, d, L, p, k, S, P, R, C = sizes(w)
+    tok = B * N * H * d * 2
+    gat = B * H * S * d * 2
+    return {
+        "pyramid": 3 * B * R * H * d * 2 + 2 * B * H * P * 4,
+        "select": B * H * S * 4 + B * H * P * 4,
+        "gather": 3 * gat,
+        "scatter": tok,
+        "scatter_bwd": gat + B * H * S * 4,
+        "gather_bwd": 3 * tok,
+    }
+
+
+def write_bandwidth(dev, nbytes=1 << 30):
+    """Measured write-only bandwidth of this GPU (GB/s): a zero fill of
+    `nbytes` (torch's fill kernel, CUDA events, best of 5).  HBM sustains far
+    less writing alone than the read + write mix of a copy, so a stage that
+    mostly writes is bounded by this figure, not by the copy peak."""
+    buf = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    best = None
+    for i in range(7):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        buf.zero_()
+        b.record()
+        torch.cuda.synchronize(dev)
+        if i >= 2:
+            t = a.elapsed_time(b)
+            best = t if best is None else min(best, t)
+    del buf
+    return nbytes / (best / 1e3) / 1e9
+
+
 EXECUTED_GEMMS = {"attn_fwd": 2, "attn_bwd_dkdv": 4, "attn_bwd_dq": 3}
 
 
@@ -329,13 +364,20 @@ def run_ours(args, w, ws, rank, local):
     # ---- roofline, per stage and for the dominant kernel
     pk = peaks()
     alg = algorithmic(w)
+    wr = algorithmic_writes(w)
+    wr_gbs = write_bandwidth(dev)
     per_stage = {}
     for name, ms in stage_ms.items():
         bound, amount = alg[name]
         if bound == "hbm":
             ach = amount / (ms / 1e3) / 1e9
+            # the shortest time its bytes allow: all of them at the copy rate,
+            # or its writes at the write-only rate, whichever is longer
+            t_min = max(amount / pk["hbm"], wr[name] / wr_gbs) / 1e9 * 1e3
             per_stage[name] = {"ms": round(ms, 4), "bound": "hbm", "GB/s": round(ach, 1),
-                               "frac": round(ach / pk["hbm"], 4), "algorithmic_bytes": amount}
+                               "frac": round(ach / pk["hbm"], 4), "algorithmic_bytes": amount,
+                               "written_bytes": wr[name],
+                               "frac_rw": round(t_min / ms, 4)}
         else:
             ach = amount / (ms / 1e3) / 1e12
             one_gemm = alg["attn_fwd"][1] / 2
@@ -370,6 +412,7 @@ def run_ours(args, w, ws, rank, local):
         "heads_this_rank": H,
         "fwd_tokens_per_s": share * B * N / (fwd_ms / 1e3), "fwd_ms": fwd_ms,
         "stages": per_stage, "roofline": roof, "e2e": e2e, "gpu_launches": launches,
+        "hbm_write_only_GB/s": round(wr_gbs, 1),
         "clocks": clocks,
     }
     return line
