@@ -410,6 +410,10 @@ constexpr int Q_M = 128;   // stationary query rows
 constexpr int KV_N = 128;  // walked key rows per tile
 constexpr int KST = 3;     // stages of the walked K ring (K is held until the dQ MMAs)
 constexpr int VST = 2;     // stages of the walked V ring (V only until the dP MMAs)
+// dS goes back to the dQ MMAs in kDsGroups groups of key columns per
+// warpgroup, each on its own barrier, so the dQ MMAs of a group run while the
+// softmax still works on the next.
+constexpr int kDsGroups = 2;
 
 // warp 0 TMA, warp 1 issuer A (S), warps 2-9 softmax, warp 10 issuer B (dQ, dP)
 constexpr int kThreadsDq = 352;
@@ -430,7 +434,7 @@ struct DqBars {
   // tensor pipe first and A's fill the time B waits for the softmax.  Two
   // barriers by parity, because B may run one step ahead of A's wait.
   uint64_t qfull, kfull[KST], kempty[KST], vfull[VST], vempty[VST], sfull[2], sfree[2], dpfull,
-      dsready, dpissued[2], done;
+      dsready[kDsGroups], dpissued[2], done;
   uint32_t tmem_base;
 };
 
@@ -438,7 +442,8 @@ struct DqBars {
 // first 32 columns of each warpgroup's 64), dQ 384.
 //
 // Issuer A computes S(j) = Q K(j)^T into the S buffer j % 2 as soon as the
-// softmax has read S(j - 2); issuer B runs dQ += dS(j - 1) K(j - 1), then
+// softmax has read S(j - 2); issuer B runs dQ += dS(j - 1) K(j - 1) (group
+// by group, as the softmax hands dS back in kDsGroups groups of keys), then
 // dP(j) = dO V(j)^T (in issue order, so dP(j) overwrites dS(j - 1) only
 // after the dQ MMAs that read it).  The softmax turns S(j) into P in
 // registers while B's MMAs run, then dP(j) into dS.  LSE and D are
@@ -477,7 +482,7 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
       mbar_init(&bars->sfree[s], kSoftmax);
     }
     mbar_init(&bars->dpfull, 1);
-    mbar_init(&bars->dsready, kSoftmax);
+    for (int g = 0; g < kDsGroups; ++g) mbar_init(&bars->dsready[g], kSoftmax);
     mbar_init(&bars->dpissued[0], 1);
     mbar_init(&bars->dpissued[1], 1);
     mbar_init(&bars->done, 1);
@@ -544,15 +549,25 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
     bool ok = mbar_wait_w(&bars->qfull, 0, status, 35);
     for (int j = 0; ok && j <= n_kv; ++j) {
       if (j > 0) {
+        // group by group as the softmax hands dS back: group g is key steps
+        // ks = 4 h + c of both warpgroups h, c in [g, g + 1) * 4 / kDsGroups
         const int sp = (j - 1) % KST;
-        if (!mbar_wait_w(&bars->dsready, (j - 1) & 1, status, 36)) { ok = false; break; }
-        tc_fence_after();
         const uint32_t kb = sK + sp * KV_N * HD * 2;
 #pragma unroll
-        for (int ks = 0; ks < KV_N / 16; ++ks)
-          mma_bf16_ts_w(tmem + 384, tmem + 256 + (ks >> 2) * 64 + (ks & 3) * 8,
-                        sdesc_sw128(kb + ks * 16 * 128, KV_N * 128, 1024), idG,
-                        (j > 1 || ks > 0) ? 1u : 0u);
+        for (int g = 0; g < kDsGroups; ++g) {
+          if (!mbar_wait_w(&bars->dsready[g], (j - 1) & 1, status, 36)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+            for (int c = g * (4 / kDsGroups); c < (g + 1) * (4 / kDsGroups); ++c) {
+              const int ks = 4 * hh + c;
+              mma_bf16_ts_w(tmem + 384, tmem + 256 + hh * 64 + c * 8,
+                            sdesc_sw128(kb + ks * 16 * 128, KV_N * 128, 1024), idG,
+                            (j > 1 || ks > 0) ? 1u : 0u);
+            }
+        }
+        if (!ok) break;
         mma_commit_w(&bars->kempty[sp]);
       }
       if (j == n_kv) break;
@@ -639,11 +654,13 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
         // chunk ch's packed dS covers fp32 columns 8 ch .. 8 ch + 7, all
         // read by the loads of chunks <= ch, which have completed
         tmem_st8(cP + ch * 8, dk);
+        if ((ch + 1) % (4 / kDsGroups) == 0) {       // group complete: hand it back
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&bars->dsready[ch / (4 / kDsGroups)]);
+        }
         if (ch < 3) tmem_ld_wait();
       }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&bars->dsready);
     }
     if (ok && mbar_wait(&bars->done, 0, status, 40)) {
       tc_fence_after();
