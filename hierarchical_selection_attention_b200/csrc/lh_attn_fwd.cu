@@ -37,8 +37,9 @@
 // either the shard's own block (causal, as above) or an earlier shard's
 // block (`full`: every key visible; keys past S masked).  Partial results
 // merge by log-sum-exp into fp32 accumulators, in base 2:
-//   lse2 = log2(2^a + 2^b),  O = O_a 2^(a - lse2) + O_b 2^(b - lse2)
-// with a the accumulated and b this block's lse2 and O_a, O_b normalised.
+//   lse2 = log2(2^u + 2^w),  O = O_u 2^(u - lse2) + O_w 2^(w - lse2)
+// with u the accumulated and w this block's lse2, and O_u, O_w their
+// normalised outputs.
 // `first` writes the accumulators without reading them; `last` writes the
 // bf16 output and natural-log LSE instead of them.  first && last is the
 // plain single-block attention.
